@@ -1,0 +1,75 @@
+"""Shared tolerance checks and row samplers for the GPU parity tests.
+
+Tolerances (stated in the design notes and applied everywhere):
+
+* fp32 path: max |gpu - oracle| <= 1e-5 (unnormalised).
+* bf16 path: rel-L2 = ||gpu - oracle|| / ||oracle|| <= 5e-3, and
+  max over elements of (|gpu - oracle| - 2^-8 |oracle|) <= 1e-2 * rms(oracle):
+  the max-abs bound in units of the oracle's RMS, after allowing the half
+  unit-in-the-last-place of the final bf16 output cast (2^-8 relative),
+  which alone exceeds 1e-2 absolute once |o| > 2.56.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BF16_REL_L2 = 5e-3
+BF16_MAX_NORM = 1e-2
+F32_MAX_ABS = 1e-5
+
+
+def to_np(t) -> np.ndarray:
+    import torch
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().numpy().astype(np.float64)
+    return np.asarray(t, dtype=np.float64)
+
+
+def bf16_errors(got, ref):
+    got, ref = to_np(got), to_np(ref)
+    diff = got - ref
+    nref = np.linalg.norm(ref)
+    rel_l2 = np.linalg.norm(diff) / max(nref, 1e-30)
+    rms = np.sqrt(np.mean(ref * ref)) if ref.size else 0.0
+    excess = np.max(np.abs(diff) - 2.0 ** -8 * np.abs(ref)) if ref.size else 0.0
+    max_norm = max(excess, 0.0) / max(rms, 1e-30)
+    return rel_l2, max_norm, float(np.max(np.abs(diff))) if ref.size else 0.0
+
+
+def assert_bf16_close(got, ref, what=""):
+    rel_l2, max_norm, max_abs = bf16_errors(got, ref)
+    assert np.all(np.isfinite(to_np(got))), f"{what}: non-finite output"
+    assert rel_l2 <= BF16_REL_L2 and max_norm <= BF16_MAX_NORM, \
+        f"{what}: rel_l2={rel_l2:.3e} max_norm={max_norm:.3e} max_abs={max_abs:.3e}"
+    return rel_l2, max_norm
+
+
+def assert_f32_close(got, ref, what="", tol=F32_MAX_ABS):
+    got, ref = to_np(got), to_np(ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    assert err <= tol, f"{what}: max abs err {err:.3e} > {tol:.1e}"
+    return err
+
+
+def sample_rows(B, H, N, window, n_random=256, seed=0, tile=128):
+    """(b, h, i) rows: the first rows (partial windows), rows around every
+    tile edge near the start and end, the last row, and random rows."""
+    rng = np.random.default_rng(seed)
+    picks = set()
+    firsts = list(range(min(N, 3))) + [min(N - 1, window - 1), min(N - 1, window), min(N - 1, 2 * window - 1)]
+    edges = []
+    for e in list(range(tile, min(N, 4 * tile + 1), tile)) + [N - tile, N - 1]:
+        for di in (-1, 0, 1):
+            if 0 <= e + di < N:
+                edges.append(e + di)
+    for b in range(B):
+        for h in range(H):
+            for i in firsts + edges[:6]:
+                if rng.random() < 0.35:
+                    picks.add((b, h, int(i)))
+    for _ in range(n_random):
+        picks.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(N))))
+    picks.add((B - 1, H - 1, N - 1))
+    picks.add((0, 0, 0))
+    return np.array(sorted(picks), dtype=np.int64)

@@ -1,0 +1,151 @@
+"""GPU ring-buffer decode parity against the oracle's own fp64 ring, through the C ABI."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sliding_window_sigmoid_b200 import binding, inputs
+from tests.helpers import assert_bf16_close, assert_f32_close, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _sync_ok():
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+
+
+@pytest.mark.parametrize("mode,w,s", [(0, 7, 0), (1, 7, 2), (0, 5, 3), (1, 1, 0), (1, 64, 4)])
+def test_f32_decode_every_step_from_position_zero(mode, w, s):
+    B, H, Hkv, d, steps, base = 2, 4, 2, 32, 23, 1e4
+    sl = inputs.balanced_alibi_slopes(H) if mode == 0 else None
+    gpu = binding.RingCache(B, H, Hkv, d, w, s, mode=mode, slopes=sl, rope_base=base,
+                            dtype=torch.float32, device=DEV)
+    ref = oracle.RingCache(B, Hkv, d, w, s, base)
+    for t in range(steps):
+        q, kn, vn = inputs.decode_step_inputs(B, H, Hkv, d, t, dtype=torch.float32)
+        pos = torch.full((B,), t, dtype=torch.int64)
+        o = gpu.step(q.to(DEV), kn.to(DEV), vn.to(DEV), pos.to(DEV))
+        _sync_ok()
+        r = ref.step(q.numpy(), kn.numpy(), vn.numpy(), pos.numpy(), mode=mode,
+                     slopes=None if sl is None else sl.numpy())
+        assert_f32_close(o, r, f"step {t}")
+
+
+def _decode_probe(dtype, w, s, p0, n_fill, steps):
+    # q = 0 and slopes 0 give every valid slot the weight 1/2; the value of
+    # position p carries the bits of p in channels 0..16 and a 1 in channel 17,
+    # so 2*o counts the positions in the key set, bit by bit: exact integers.
+    B, H, Hkv, d = 2, 2, 1, 64
+    gpu = binding.RingCache(B, H, Hkv, d, w, s, mode=0, slopes=None, rope_base=1e4, dtype=dtype,
+                            device=DEV)
+
+    def vrow(p):
+        x = torch.zeros(d)
+        for c in range(17):
+            x[c] = (p >> c) & 1
+        x[17] = 1.0
+        return x
+
+    if s > 0:   # sinks come from a prefill of positions 0..s-1
+        ks = torch.zeros(B, s, Hkv, d, dtype=dtype)
+        vs = torch.stack([vrow(p) for p in range(s)]).to(dtype)[None, :, None, :].expand(B, s, Hkv, d).contiguous()
+        gpu.fill(ks.to(DEV), vs.to(DEV), 0)
+    if n_fill:
+        kf = torch.zeros(B, n_fill, Hkv, d, dtype=dtype)
+        vf = torch.stack([vrow(p0 + t) for t in range(n_fill)]).to(dtype)[None, :, None, :]
+        vf = vf.expand(B, n_fill, Hkv, d).contiguous()
+        gpu.fill(kf.to(DEV), vf.to(DEV), p0)
+    for t in range(steps):
+        P = p0 + n_fill + t
+        q = torch.zeros(B, H, d, dtype=dtype)
+        kn = torch.zeros(B, Hkv, d, dtype=dtype)
+        vn = vrow(P).to(dtype)[None, None, :].expand(B, Hkv, d).contiguous()
+        o = gpu.step(q.to(DEV), kn.to(DEV), vn.to(DEV), torch.full((B,), P, dtype=torch.int64, device=DEV))
+        _sync_ok()
+        got = 2.0 * to_np(o)[:, :, :18]
+        keys = [j for j in range(P + 1) if oracle.in_keyset(P, j, w, s)]
+        want = np.array([sum((j >> c) & 1 for j in keys) for c in range(17)] + [len(keys)], float)
+        for b in range(B):
+            for h in range(H):
+                np.testing.assert_array_equal(got[b, h], want, err_msg=f"pos {P}")
+        # value cache: slot P mod w holds position P's value, bit for bit
+        np.testing.assert_array_equal(to_np(gpu.v_cache[0, 0, P % w]), to_np(vn[0, 0]))
+
+
+_F32, _BF16 = torch.float32, torch.bfloat16
+
+
+# bf16 outputs hold the half-counts exactly while they stay <= 128 (key sets
+# of at most 256 positions), so the larger rings run on the fp32 path only.
+@pytest.mark.parametrize("dtype,w,s,p0,n_fill,steps", [
+    (_F32, 8, 0, 0, 0, 20), (_BF16, 8, 0, 0, 0, 20),        # partial ring from 0, wraparound
+    (_F32, 8, 3, 3, 9, 12), (_BF16, 8, 3, 3, 9, 12),        # sinks, fill past the window
+    (_F32, 64, 4, 0, 100, 70), (_BF16, 64, 4, 0, 100, 70),  # sinks overlap the window early on
+    (_F32, 1030, 2, 1000, 1100, 3),                         # several slot chunks, ragged last
+    (_BF16, 250, 2, 1000, 260, 3),
+    (_F32, 1, 2, 2, 5, 4), (_BF16, 1, 2, 2, 5, 4),          # window of one slot
+])
+def test_decode_index_probe_bit_exact(dtype, w, s, p0, n_fill, steps):
+    _decode_probe(dtype, w, s, p0, n_fill, steps)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_bf16_decode_equals_oracle_ring_and_forward_row(mode):
+    B, H, Hkv, d, w, s, N = 2, 8, 2, 128, 64, 4, 300
+    base = 1e4 if mode == 0 else 5e5
+    sl = inputs.balanced_alibi_slopes(H) if mode == 0 else None
+    q, k, v = inputs.qkv(B, N, H, Hkv, d, seed=17, dtype=torch.bfloat16)
+    P = 250
+    gpu = binding.RingCache(B, H, Hkv, d, w, s, mode=mode, slopes=sl, rope_base=base, device=DEV)
+    gpu.fill(k[:, :P].contiguous().to(DEV), v[:, :P].contiguous().to(DEV), 0)
+    ref = oracle.RingCache(B, Hkv, d, w, s, base)
+    f = lambda t: t.float().numpy()
+    ref.fill(f(k[:, :P]), f(v[:, :P]), 0)
+    o_fwd, _ = oracle.swat_fwd(f(q), f(k), f(v), window=w, n_sink=s, mode=mode,
+                               slopes=None if sl is None else sl.numpy(), rope_base=base)
+    for p in range(P, N):
+        pos = torch.full((B,), p, dtype=torch.int64, device=DEV)
+        o = gpu.step(q[:, p].contiguous().to(DEV), k[:, p].contiguous().to(DEV),
+                     v[:, p].contiguous().to(DEV), pos)
+        _sync_ok()
+        r = ref.step(f(q[:, p]), f(k[:, p]), f(v[:, p]), np.full(B, p), mode=mode,
+                     slopes=None if sl is None else sl.numpy())
+        assert_bf16_close(o, r, f"decode {p}")
+        np.testing.assert_allclose(r, o_fwd[:, p], atol=1e-9)   # oracle ring == oracle forward row
+
+
+@pytest.mark.parametrize("wl", [inputs.DECODE_SIGMOID, inputs.DECODE_SOFTMAX], ids=lambda w: w.name)
+def test_full_size_ring_decode_sampled_sequences(wl):
+    # batch 64, 32/8 heads, d 128, window 4096: ring prefilled with positions
+    # 28672..32767 (and sinks 0..3), then steps from position 32768 (which
+    # already wraps onto slot 0). The oracle keeps full rings for b in {0, 37, 63}.
+    B, H, Hkv, d, w, s = wl.B, wl.H, wl.Hkv, wl.d, wl.window, wl.n_sink
+    sl = wl.slope_tensor()
+    p_start = wl.start_pos
+    kf = inputs.normal((B, w, Hkv, d), 501)
+    vf = inputs.normal((B, w, Hkv, d), 502)
+    gpu = binding.RingCache(B, H, Hkv, d, w, s, mode=wl.mode, slopes=sl, rope_base=wl.rope_base,
+                            device=DEV)
+    bsel = [0, 37, 63]
+    ref = oracle.RingCache(len(bsel), Hkv, d, w, s, wl.rope_base)
+    f = lambda t: t.float().numpy()
+    if s > 0:
+        ks = inputs.normal((B, s, Hkv, d), 503)
+        vs = inputs.normal((B, s, Hkv, d), 504)
+        gpu.fill(ks.to(DEV), vs.to(DEV), 0)
+        ref.fill(f(ks[bsel]), f(vs[bsel]), 0)
+    gpu.fill(kf.to(DEV), vf.to(DEV), p_start - w)
+    ref.fill(f(kf[bsel]), f(vf[bsel]), p_start - w)
+    for t in range(6):
+        q, kn, vn = inputs.decode_step_inputs(B, H, Hkv, d, t)
+        pos = torch.full((B,), p_start + t, dtype=torch.int64)
+        o = gpu.step(q.to(DEV), kn.to(DEV), vn.to(DEV), pos.to(DEV))
+        _sync_ok()
+        r = ref.step(f(q[bsel]), f(kn[bsel]), f(vn[bsel]), pos.numpy()[bsel], mode=wl.mode,
+                     slopes=None if sl is None else sl.numpy())
+        assert_bf16_close(o[bsel], r, f"{wl.name} step {t}")
+        assert torch.isfinite(o.float()).all()
