@@ -289,6 +289,29 @@ def run_swat(args):
                 "bwd": {"tflops": bwd_tf, "frac": bwd_tf / peak, "ms": bwd_ms}}
 
     # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, kw)
+
+    # ---- ring-buffer decode (batch 64, 32/8 heads, d 128, window 4096) ----
+    decode = {}
+    if not args.no_decode:
+        del q, k, v, do, o, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+        decode = bench_decode(args, dev, world, rank, peaks, peak_src)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_sample(8)
+    _print_line(args, rank, world, value, ms, B, H, Hkv, d, N, w, wl, roofline, cpu, e2e, clocks,
+                launches, fwd_tf, bwd_tf, decode)
+
+
+def bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, kw):
+    """Same step through the public API with host buffers: every step copies
+    Q, K, V, dO from pinned host memory and reads O, dQ, dK, dV back."""
+    import torch
+    from sliding_window_sigmoid_b200 import binding
     hq, hk, hv, hdo = [t.cpu().pin_memory() for t in (q, k, v, do)]
     ho, hdq, hdk, hdv = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, dq, dk, dv)]
     dq_in, dk_in, dv_in, ddo_in = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
@@ -322,19 +345,11 @@ def run_swat(args):
     e2e = {"value": step_flops * world * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
            "h2d_bytes_per_step": nbytes((hq, hk, hv, hdo)),
            "d2h_bytes_per_step": nbytes((ho, hdq, hdk, hdv))}
-    del hq, hk, hv, hdo, ho, hdq, hdk, hdv, dq_in, dk_in, dv_in, ddo_in
+    return e2e
 
-    # ---- ring-buffer decode (batch 64, 32/8 heads, d 128, window 4096) ----
-    decode = {}
-    if not args.no_decode:
-        del q, k, v, do, o, dq, dk, dv, ws
-        torch.cuda.empty_cache()
-        decode = bench_decode(args, dev, world, rank, peaks, peak_src)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline_sample(8)
-
+def _print_line(args, rank, world, value, ms, B, H, Hkv, d, N, w, wl, roofline, cpu, e2e, clocks,
+                launches, fwd_tf, bwd_tf, decode):
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -411,6 +426,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -172,6 +172,8 @@ class RingCache:
         self.B, self.H, self.Hkv, self.d, self.window, self.n_sink = B, H, Hkv, d, window, n_sink
         self.mode, self.rope_base, self.dtype = mode, float(rope_base), dtype
         self.device = torch.device(device)
+        if self.device.type == "cuda" and self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
         self.k_cache = torch.zeros(B, Hkv, window, d, dtype=dtype, device=self.device)
         self.v_cache = torch.zeros_like(self.k_cache)
         ns = max(n_sink, 1)

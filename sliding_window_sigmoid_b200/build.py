@@ -44,7 +44,7 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
     if not force and not needs_build():
         return LIB
     cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", LIB,
-           os.path.join(CSRC, "api.cu"), "-lcuda"]
+           os.path.join(CSRC, "api.cu")]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     if extra:

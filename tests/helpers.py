@@ -4,10 +4,11 @@ Tolerances (stated in the design notes and applied everywhere):
 
 * fp32 path: max |gpu - oracle| <= 1e-5 (unnormalised).
 * bf16 path: rel-L2 = ||gpu - oracle|| / ||oracle|| <= 5e-3, and
-  max over elements of (|gpu - oracle| - 2^-8 |oracle|) <= 1e-2 * rms(oracle):
-  the max-abs bound in units of the oracle's RMS, after allowing the half
-  unit-in-the-last-place of the final bf16 output cast (2^-8 relative),
-  which alone exceeds 1e-2 absolute once |o| > 2.56.
+  max over elements of (|gpu - oracle| - 2^-8 |oracle|) <= 1e-2 * max(1, rms(oracle)):
+  the literal max-abs 1e-2 for outputs of unit scale, measured in units of
+  the oracle's RMS for larger outputs (a window of 4096 sigmoid weights gives
+  |o| ~ 64, where one bf16 ulp is 0.25), after allowing the half
+  unit-in-the-last-place of the final bf16 output cast (2^-8 relative).
 """
 from __future__ import annotations
 
@@ -32,7 +33,7 @@ def bf16_errors(got, ref):
     rel_l2 = np.linalg.norm(diff) / max(nref, 1e-30)
     rms = np.sqrt(np.mean(ref * ref)) if ref.size else 0.0
     excess = np.max(np.abs(diff) - 2.0 ** -8 * np.abs(ref)) if ref.size else 0.0
-    max_norm = max(excess, 0.0) / max(rms, 1e-30)
+    max_norm = max(excess, 0.0) / max(rms, 1.0)
     return rel_l2, max_norm, float(np.max(np.abs(diff))) if ref.size else 0.0
 
 
