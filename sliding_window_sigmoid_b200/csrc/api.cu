@@ -87,6 +87,7 @@ int swat_attn_fwd(const void *q, const void *k, const void *v, void *o, float *l
     if ((lse && !aligned16(lse)) || (slopes && (reinterpret_cast<uintptr_t>(slopes) & 3u)))
         return SWAT_ERR_INVALID_ARG;
 
+    if (window > N) window = N;   // a window of N already covers every earlier key
     if (dtype == SWAT_BF16) {
         swat::TcFwdArgs a{};
         a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.slopes = slopes;
@@ -133,6 +134,7 @@ int swat_attn_bwd(const void *q, const void *k, const void *v, const void *o, co
     for (const void *p : ptrs) if (!aligned16(p)) return SWAT_ERR_INVALID_ARG;
     if (o && !aligned16(o)) return SWAT_ERR_INVALID_ARG;
 
+    if (window > N) window = N;
     swat::BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;
     a.dq = dq; a.dk = dk; a.dv = dv; a.Dws = (float *)workspace; a.slopes = slopes;

@@ -24,6 +24,7 @@
 // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D). P_b aliases the
 // first 64 columns of S_b (bf16 pairs).
 #pragma once
+#include <algorithm>
 #include "common.cuh"
 #include "sm100.cuh"
 #include "fwd_simt.cuh"
@@ -35,30 +36,44 @@ using TcFwdArgs = FwdArgs;
 
 template <int D>
 struct FwdTcCfg {
-    static constexpr int BM = 128, BN = 128;
-    static constexpr int NST = (D == 64) ? 3 : 2;            // K/V pipeline stages
     static constexpr int TILE_BYTES = 128 * D * 2;            // one 128-row bf16 tile
     static constexpr int HALF_BYTES = 128 * 128;              // one 64-column SW128 box
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + TILE_BYTES;
-    static constexpr int OFF_V = OFF_K + NST * TILE_BYTES;
-    static constexpr int OFF_W = OFF_V + NST * TILE_BYTES;    // float2 [D/2][32]
-    static constexpr int OFF_E = OFF_W + (D / 2) * 32 * 8;    // float2 [2][4][D/2]
-    static constexpr int OFF_TH = OFF_E + 2 * 4 * (D / 2) * 8;   // double [D/2]
+    static constexpr int NSLOT = (D == 64) ? 5 : 2;           // K/V ring slots
+    static constexpr int OFF_Q = 0;                           // two Q buffers
+    static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + NSLOT * TILE_BYTES;
+    static constexpr int OFF_E = OFF_V + NSLOT * TILE_BYTES;  // float2 [2][D/2]
+    static constexpr int OFF_TH = OFF_E + 2 * (D / 2) * 8;    // double [D/2]
     static constexpr int OFF_BAR = OFF_TH + (D / 2) * 8;
-    static constexpr int NBAR = 2 + 4 * NST + 4 + 3;
+    static constexpr int NBAR = 6 + 4 * NSLOT + 6 + 4 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;         // + slack for 1024-B alignment
-    static constexpr int THREADS = 320;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t COL_O = 256;
+    static constexpr int NSB = (D == 64) ? 3 : 2;              // S buffers of 128 columns
+    static constexpr uint32_t COL_O = NSB * 128;              // O0 at COL_O, O1 at COL_O + D
 };
 
-constexpr int FWD_ACT_WARP0 = 0, FWD_PREP_WARP0 = 4, FWD_MMA_WARP = 8, FWD_TMA_WARP = 9;
+// Warp roles. Sigmoid mode runs two activation warpgroups that take the S
+// tiles in turn (even steps / odd steps), so one computes while the other
+// waits for its next tile; softmax mode keeps one, because a row's running
+// maximum and sum must live in one thread.
+// Warps 0 and 1 issue MMAs and TMA copies: the scheduler favours older
+// (lower-numbered) warps, and these two threads pace everything else.
+// Warps 2-3 are idle; activation warpgroups start at warp 4 so that warp w
+// owns TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31.
+template <int MODE>
+struct FwdRoles {
+    static constexpr int ACT_WG = (MODE == SWAT_MODE_SIGMOID_) ? 2 : 1;
+    static constexpr int MMA_WARP = 0;
+    static constexpr int TMA_WARP = 1;
+    static constexpr int ACT_WARP0 = 4;
+    static constexpr int PREP_WARP0 = ACT_WARP0 + 4 * ACT_WG;
+    static constexpr int THREADS = 32 * (PREP_WARP0 + 4);
+};
 constexpr int FWD_PREP_BAR = 1;   // named barrier of the 128 prep threads
 
-// Key tiles of a query tile: optional sink tile (keys 0..127) when the band
-// starts above it, then the band tiles from floor(max(0,i0-w+1)/128) to the
+// Key tiles of a query tile: an optional sink tile (keys 0..127) when the band
+// starts above it, then the band tiles from floor(max(0, i0-w+1)/128) to the
 // tile holding min(N-1, i0+127).
 struct TileRange {
     int n_tiles, has_sink, j0_first;
@@ -78,6 +93,150 @@ __device__ __forceinline__ int fwd_tile_j0(const TileRange &r, int t)
 {
     return (r.has_sink && t == 0) ? 0 : r.j0_first + (t - r.has_sink) * 128;
 }
+
+// ---------------------------------------------------------------------------
+// Static schedule of a persistent CTA. Work items are (b, kv head, query
+// tile, head in group), in that order (group heads fastest), so consecutive
+// items share most key tiles: a query tile slides the window by one tile and
+// the heads of a group read the same K/V. Each CTA takes a contiguous range
+// of items. Every role walks the same sequence of steps (item, key tile):
+// - RESIDENT mode (the band of a query tile fits the ring): band tile jt of a
+//   sequence lives in ring slot jt mod R and is loaded (and rotated) once,
+//   when the first item of the range needs it, and released after the last
+//   item that needs it; the sink tile has a slot of its own.
+// - STREAMING mode: every step loads its tile into the next ring slot.
+// ---------------------------------------------------------------------------
+struct FwdItem {
+    int valid, b, kvh, h, i0, seq, lo, hi, n_tiles, has_sink;
+};
+
+struct FwdStep {
+    int k, first, last, step;                // local item index, first/last tile of the item, global step
+    int b, kvh, h, i0, j0;
+    int slot, par, is_new, need_release, last_use;
+};
+
+struct FwdSched {
+    int N, window, n_sink, Hkv, G, nQT;
+    int u, u_end, u_begin;                   // item indices fit 32 bits (checked on the host)
+    int nslot, r_band, resident;
+    int t, k, step, stream_slot, band_slot;
+    int next_load, seq_lo0, seq_slot0;       // RESIDENT mode: round-robin load pointer, slot of the sequence's first tile
+    uint32_t cur_par, loaded;
+    FwdItem cur, nxt;
+    int p_valid, p_seq, p_lo, p_hi, p_sink;
+
+    __device__ FwdItem item(int uu) const
+    {
+        FwdItem it;
+        it.valid = (uu >= u_begin && uu < u_end);
+        if (!it.valid) { it.seq = -1; it.lo = it.hi = it.has_sink = 0; return it; }
+        const unsigned v = (unsigned)uu;
+        const unsigned g = v % (unsigned)G, r = v / (unsigned)G;
+        const unsigned qt = r % (unsigned)nQT, sq = r / (unsigned)nQT;
+        it.seq = (int)sq;
+        it.kvh = (int)(sq % (unsigned)Hkv);
+        it.b = (int)(sq / (unsigned)Hkv);
+        it.h = it.kvh * G + (int)g;
+        it.i0 = (int)qt * 128;
+        const TileRange tr = fwd_tile_range(it.i0, N, window, n_sink);
+        it.lo = tr.j0_first / 128;
+        it.hi = min(N - 1, it.i0 + 127) / 128;
+        it.n_tiles = tr.n_tiles;
+        it.has_sink = tr.has_sink;
+        return it;
+    }
+
+    // Band tiles of one sequence are loaded in increasing order into
+    // consecutive slots, starting at the least recently loaded slot when the
+    // sequence starts in this CTA; so a load always evicts the tile loaded
+    // r_band loads earlier, whose last use lies several steps back.
+    __device__ void start_item()
+    {
+        t = 0;
+        if (!resident || !cur.valid) return;
+        if (!(p_valid && p_seq == cur.seq)) {
+            seq_lo0 = cur.lo;
+            seq_slot0 = next_load;
+        }
+        band_slot = (seq_slot0 + (cur.lo - seq_lo0)) % r_band;
+    }
+
+    __device__ void init(const FwdArgs &a, int nslot_, int cta, int ncta)
+    {
+        N = a.N; window = a.window; n_sink = a.n_sink; Hkv = a.Hkv; G = a.H / a.Hkv;
+        nQT = (a.N + 127) / 128;
+        const long long U = (long long)a.B * Hkv * nQT * G;
+        u_begin = (int)(U * cta / ncta);
+        u_end = (int)(U * (cta + 1) / ncta);
+        u = u_begin;
+        nslot = nslot_;
+        const long long wmax = min((long long)nQT, ((long long)window + 126) / 128 + 1);
+        r_band = n_sink > 0 ? nslot - 1 : nslot;
+        resident = (wmax <= r_band) ? 1 : 0;
+        k = 0; step = 0; stream_slot = 0; cur_par = 0; loaded = 0;
+        next_load = 0; seq_lo0 = 0; seq_slot0 = 0;
+        p_valid = 0; p_seq = -1; p_lo = p_hi = p_sink = 0;
+        cur = item(u);
+        nxt = item(u + 1);
+        start_item();
+    }
+
+    __device__ __forceinline__ bool next_step(FwdStep &s)
+    {
+        if (u >= u_end) return false;
+        s.k = k; s.step = step;
+        s.first = (t == 0);
+        s.last = (t == cur.n_tiles - 1);
+        s.b = cur.b; s.kvh = cur.kvh; s.h = cur.h; s.i0 = cur.i0;
+        const bool sink = cur.has_sink && t == 0;
+        const int jt = sink ? 0 : cur.lo + t - cur.has_sink;
+        s.j0 = jt * 128;
+        int slot, is_new, last_use;
+        if (resident) {
+            const bool same_prev = p_valid && p_seq == cur.seq;
+            const bool same_next = nxt.valid && nxt.seq == cur.seq;
+            if (sink) {
+                slot = r_band;
+                is_new = !(same_prev && p_sink);
+                last_use = !(same_next && nxt.has_sink);
+            } else {
+                slot = band_slot;
+                band_slot = (band_slot + 1 == r_band) ? 0 : band_slot + 1;
+                is_new = !(same_prev && p_lo <= jt && jt <= p_hi);
+                last_use = !(same_next && jt >= nxt.lo);
+                if (is_new) next_load = band_slot;   // the slot after the one just loaded
+            }
+        } else {
+            slot = stream_slot;
+            stream_slot = (stream_slot + 1 == nslot) ? 0 : stream_slot + 1;
+            is_new = 1;
+            last_use = 1;
+        }
+        const uint32_t bit = 1u << slot;
+        if (is_new) {
+            const uint32_t was = loaded & bit;
+            const uint32_t par = was ? ((cur_par & bit) ^ bit) : 0u;
+            cur_par = (cur_par & ~bit) | par;
+            loaded |= bit;
+            s.par = par ? 1 : 0;
+            s.need_release = was ? 1 : 0;
+        } else {
+            s.par = (cur_par & bit) ? 1 : 0;
+            s.need_release = 0;
+        }
+        s.slot = slot; s.is_new = is_new; s.last_use = last_use;
+        ++step;
+        if (++t == cur.n_tiles) {
+            ++k; ++u;
+            p_valid = cur.valid; p_seq = cur.seq; p_lo = cur.lo; p_hi = cur.hi; p_sink = cur.has_sink;
+            cur = nxt;
+            nxt = item(u + 1);
+            start_item();
+        }
+        return true;
+    }
+};
 
 __device__ __forceinline__ bool named_bar_or(int id, int n, bool v)
 {
@@ -118,80 +277,262 @@ __device__ __forceinline__ float2 rope_cs(double pos_theta)
 }
 
 // Rotate a 128-row tile in place (SW128 layout, D/64 boxes of [128 rows][128 B]).
-// Thread (w, l) owns row r = 32 w + l. The angle of row r, pair t is
-// (pos0 + 32 w + l) theta_t = base angle Eb[w][t] plus table angle W[t][l].
+// Thread tau owns 16-byte chunk c = tau % (D/8) of rows r0, r0 + RS, ...
+// (r0 = tau / (D/8), RS = 1024 / D), i.e. the four pairs t = 4c .. 4c+3 of
+// D/8 rows. Their rotation (pos0 + r) theta_t starts from the tile base
+// E0[t] = e^{i pos0 theta_t} times the thread's own e^{i r0 theta_t} and
+// advances by e^{i RS theta_t} from row to row (complex products in fp32).
+struct RotThread {
+    float w0c[4], w0s[4], stc[4], sts[4];   // e^{i r0 theta_t}, e^{i RS theta_t}
+};
+
 template <int D>
-__device__ __forceinline__ void rope_rotate_tile(uint8_t *tile, const float2 *W, const float2 *Eb, int w,
-                                                 int l)
+__device__ __forceinline__ void rope_rotate_tile(uint8_t *tile, const float2 *E0, const RotThread &R, int tau)
 {
-    const int r = 32 * w + l;
+    constexpr int CPR = D / 8, RS = 128 / CPR;
+    const int c = tau % CPR, r0 = tau / CPR;
+    float cc[4], ss[4];
 #pragma unroll
-    for (int hh = 0; hh < D / 64; ++hh) {
-        uint8_t *rowp = tile + hh * 16384 + r * 128;
+    for (int q = 0; q < 4; ++q) {
+        const float2 e = E0[4 * c + q];
+        cc[q] = e.x * R.w0c[q] - e.y * R.w0s[q];
+        ss[q] = e.y * R.w0c[q] + e.x * R.w0s[q];
+    }
+    uint8_t *base = tile + (c / 8) * 16384;
+    constexpr int BATCH = 8;   // rows loaded ahead of their arithmetic
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint4 *p = reinterpret_cast<uint4 *>(rowp + ((c ^ (r & 7)) << 4));
-            uint4 v = *p;
-            uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    for (int kb = 0; kb < CPR; kb += BATCH) {
+    uint4 v[BATCH];
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int t = hh * 32 + 4 * c + qq;
-                const float2 e = Eb[w * (D / 2) + t];
-                const float2 wt = W[t * 32 + l];
-                const float cs = e.x * wt.x - e.y * wt.y;
-                const float sn = e.y * wt.x + e.x * wt.y;
-                const float x0 = sm100::bf16lo(w4[qq]), x1 = sm100::bf16hi(w4[qq]);
-                w4[qq] = sm100::pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
-            }
-            *p = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    for (int k = 0; k < BATCH; ++k) {
+        const int r = r0 + RS * (kb + k);
+        v[k] = *reinterpret_cast<const uint4 *>(base + r * 128 + (((c % 8) ^ (r & 7)) << 4));
+    }
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+        const int r = r0 + RS * (kb + k);
+        uint32_t w4[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float x0 = sm100::bf16lo(w4[q]), x1 = sm100::bf16hi(w4[q]);
+            w4[q] = sm100::pack_bf16x2(x0 * cc[q] - x1 * ss[q], x0 * ss[q] + x1 * cc[q]);
+            const float nc = cc[q] * R.stc[q] - ss[q] * R.sts[q];
+            ss[q] = ss[q] * R.stc[q] + cc[q] * R.sts[q];
+            cc[q] = nc;
         }
+        *reinterpret_cast<uint4 *>(base + r * 128 + (((c % 8) ^ (r & 7)) << 4)) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
     }
 }
 
+// Valid key columns of one query row inside a 128-key tile: c in [lo, hi]
+// (the window part: 0 <= i - j < window with hi = i - j0) or c < sh (sinks,
+// which also need j <= i). Evaluated without branches.
+struct RowMask {
+    int lo, hi, sh;
+};
+
+__device__ __forceinline__ RowMask row_mask(int rd, int j0, int window, int n_sink)
+{
+    RowMask m;
+    m.lo = rd - window + 1;
+    m.hi = rd;
+    m.sh = min(n_sink - j0, rd + 1);
+    return m;
+}
+
+__device__ __forceinline__ bool col_valid(const RowMask &m, int c)
+{
+    return ((c >= m.lo) & (c <= m.hi)) | (c < m.sh);
+}
+
+// Sigmoid weights of one S tile (TMEM, one row per thread) into bf16 P over
+// the first 64 columns of the same buffer. sigma(x) = 0.5 + 0.5 tanh(x / 2)
+// with x = s/sqrt(d) + slope (i - j); rd = i - j0.
+template <bool MASKED>
+__device__ __forceinline__ void sigmoid_chunk(const uint32_t (&v)[16], uint32_t (&pk)[8], sm100::f2 bias,
+                                              sm100::f2 step2, sm100::f2 hs2, const RowMask &mk, int c0)
+{
+    const sm100::f2 half2 = {0.5f, 0.5f};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const sm100::f2 acc = {__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])};
+        const sm100::f2 x = sm100::fma2(acc, hs2, bias);
+        bias = sm100::add2(bias, step2);
+        const sm100::f2 th = {sm100::tanh_approx(x.x), sm100::tanh_approx(x.y)};
+        sm100::f2 p = sm100::fma2(th, half2, half2);
+        if (MASKED) {
+            p.x = col_valid(mk, c0 + 2 * e) ? p.x : 0.f;
+            p.y = col_valid(mk, c0 + 2 * e + 1) ? p.y : 0.f;
+        }
+        pk[e] = sm100::pack_bf16x2(p.x, p.y);
+    }
+}
+
+// One 16-column chunk of P: skipped (P = 0) when no key of the chunk is
+// valid for any row of the warp, masked per element when some are not.
+template <bool MASKED>
+__device__ __forceinline__ void sigmoid_chunk_any(const uint32_t (&v)[16], uint32_t s_addr, int c0,
+                                                  sm100::f2 step2, sm100::f2 hs2, sm100::f2 nh2,
+                                                  sm100::f2 hb2, const RowMask &mk, int rd_w0, int window,
+                                                  int sink_cols)
+{
+    uint32_t pk[8];
+    const sm100::f2 cpair = {(float)c0, (float)(c0 + 1)};
+    const sm100::f2 bias = sm100::fma2(cpair, nh2, hb2);   // 0.5 slope (i - j) for columns c0, c0+1
+    if (MASKED) {
+        const bool all_in = (c0 >= rd_w0 + 32 - window) && (c0 + 15 <= rd_w0);
+        const bool all_out = ((c0 > rd_w0 + 31) || (c0 + 15 < rd_w0 - window + 1)) && (c0 >= sink_cols);
+        if (all_out) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[e] = 0u;
+        } else if (all_in) {
+            sigmoid_chunk<false>(v, pk, bias, step2, hs2, mk, c0);
+        } else {
+            sigmoid_chunk<true>(v, pk, bias, step2, hs2, mk, c0);
+        }
+    } else {
+        sigmoid_chunk<false>(v, pk, bias, step2, hs2, mk, c0);
+    }
+    sm100::tmem_st8(s_addr + (c0 >> 1), pk);
+}
+
+// Sigmoid weights of one S tile (TMEM, one row per thread) into bf16 P over
+// the first 64 columns of the same buffer. sigma(x) = 0.5 + 0.5 tanh(x / 2)
+// with x = s/sqrt(d) + slope (i - j); rd = i - j0 for this thread's row and
+// rd_w0 for the warp's first row. On edge tiles each 16-column chunk is
+// classified for the whole warp: every key valid, none valid (P = 0 without
+// arithmetic), or mixed (per-element mask). The chunk loop is kept rolled
+// (two chunks per iteration for the double-buffered TMEM loads) so the hot
+// code stays small in the instruction cache.
+template <bool MASKED>
+__device__ __forceinline__ void act_sigmoid_tile(uint32_t s_addr, float hs, float hsl, int rd, int rd_w0, int j0,
+                                                 int window, int n_sink)
+{
+    const RowMask mk = row_mask(rd, j0, window, n_sink);
+    const sm100::f2 hs2 = {hs, hs}, step2 = {-2.f * hsl, -2.f * hsl}, nh2 = {-hsl, -hsl};
+    const float hb0 = hsl * (float)rd;
+    const sm100::f2 hb2 = {hb0, hb0};
+    const int sink_cols = n_sink - j0;
+    uint32_t v0[16], v1[16];
+    sm100::tmem_ld16(s_addr, v0);
+    sm100::tmem_wait_ld_dep16(v0);
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+        sm100::tmem_ld16(s_addr + c0 + 16, v1);
+        sigmoid_chunk_any<MASKED>(v0, s_addr, c0, step2, hs2, nh2, hb2, mk, rd_w0, window, sink_cols);
+        sm100::tmem_wait_ld_dep16(v1);
+        if (c0 + 32 < 128) sm100::tmem_ld16(s_addr + c0 + 32, v0);
+        sigmoid_chunk_any<MASKED>(v1, s_addr, c0 + 16, step2, hs2, nh2, hb2, mk, rd_w0, window, sink_cols);
+        if (c0 + 32 < 128) sm100::tmem_wait_ld_dep16(v0);
+    }
+}
+
+// Softmax weights (log2 domain) of one S tile; returns the tile's row max
+// through `mx` in pass one and writes p = 2^(x - m_used) in pass two.
+template <bool MASKED>
+__device__ __forceinline__ float act_softmax_max(uint32_t s_addr, float sc2, float sl2, int rd, int j0,
+                                                 int window, int n_sink)
+{
+    float mx = -INFINITY;
+    const float b2 = sl2 * (float)rd;
+    const RowMask mk = row_mask(rd, j0, window, n_sink);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t v[32];
+        sm100::tmem_ld32(s_addr + 32 * k, v);
+        sm100::tmem_wait_ld_dep(v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int c = 32 * k + e;
+            float x = fmaf(__uint_as_float(v[e]), sc2, fmaf(-sl2, (float)c, b2));
+            if (MASKED) x = col_valid(mk, c) ? x : -INFINITY;
+            mx = fmaxf(mx, x);
+        }
+    }
+    return mx;
+}
+
+template <bool MASKED>
+__device__ __forceinline__ float act_softmax_p(uint32_t s_addr, float sc2, float sl2, int rd, int j0,
+                                               int window, int n_sink, float m_used)
+{
+    float lsum = 0.f;
+    const float b2 = sl2 * (float)rd;
+    const RowMask mk = row_mask(rd, j0, window, n_sink);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t v[32];
+        sm100::tmem_ld32(s_addr + 32 * k, v);
+        sm100::tmem_wait_ld_dep(v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c0 = 32 * k + 2 * e;
+            float x0 = fmaf(__uint_as_float(v[2 * e]), sc2, fmaf(-sl2, (float)c0, b2));
+            float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sc2, fmaf(-sl2, (float)(c0 + 1), b2));
+            float p0 = (m_used == -INFINITY) ? 0.f : sm100::ex2_approx(x0 - m_used);
+            float p1 = (m_used == -INFINITY) ? 0.f : sm100::ex2_approx(x1 - m_used);
+            if (MASKED) {
+                p0 = col_valid(mk, c0) ? p0 : 0.f;
+                p1 = col_valid(mk, c0 + 1) ? p1 : 0.f;
+            }
+            lsum += p0 + p1;
+            pk[e] = sm100::pack_bf16x2(p0, p1);
+        }
+        sm100::tmem_st16(s_addr + 16 * k, pk);
+    }
+    return lsum;
+}
+
 template <int D, int MODE>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(FwdRoles<MODE>::THREADS, 1)
 swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs a)
 {
     using C = FwdTcCfg<D>;
-    constexpr int NST = C::NST;
+    using RL = FwdRoles<MODE>;
+    constexpr int NS = C::NSLOT;
+    constexpr int FWD_PREP_WARP0 = RL::PREP_WARP0, FWD_MMA_WARP = RL::MMA_WARP, FWD_TMA_WARP = RL::TMA_WARP;
+    constexpr int FWD_ACT_WARP0 = RL::ACT_WARP0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem + C::OFF_Q;
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
-    float2 *sW = reinterpret_cast<float2 *>(smem + C::OFF_W);
     float2 *sE = reinterpret_cast<float2 *>(smem + C::OFF_E);
     double *sTh = reinterpret_cast<double *>(smem + C::OFF_TH);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *q_full = bars + 0, *q_ready = bars + 1;
-    uint64_t *k_full = bars + 2, *k_ready = k_full + NST, *v_full = k_ready + NST, *kv_empty = v_full + NST;
-    uint64_t *s_full = kv_empty + NST, *p_full = s_full + 2;
-    uint64_t *o_full = p_full + 2, *o_upd = o_full + 1, *drain = o_upd + 1;
+    uint64_t *q_full = bars, *q_ready = bars + 2, *q_free = bars + 4;
+    uint64_t *k_full = bars + 6, *k_ready = k_full + NS, *v_full = k_ready + NS, *release = v_full + NS;
+    constexpr int NSB = C::NSB;
+    uint64_t *s_full = release + NS, *p_full = s_full + NSB;
+    uint64_t *o_full = p_full + NSB, *o_free = o_full + 2;
+    uint64_t *o_upd = o_free + 2, *drain = o_upd + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int G = a.H / a.Hkv, kvh = h / G;
-    const int i0 = qt * 128;
-    const TileRange tr = fwd_tile_range(i0, a.N, a.window, a.n_sink);
-    const int T = tr.n_tiles;
 
     if (threadIdx.x == 0) {
-        sm100::mbar_init(q_full, 1);
-        sm100::mbar_init(q_ready, 128);
-        for (int s = 0; s < NST; ++s) {
-            sm100::mbar_init(k_full + s, 1);
-            sm100::mbar_init(k_ready + s, 128);
-            sm100::mbar_init(v_full + s, 1);
-            sm100::mbar_init(kv_empty + s, 1);
-        }
         for (int s = 0; s < 2; ++s) {
+            sm100::mbar_init(q_full + s, 1);
+            sm100::mbar_init(q_ready + s, 128);
+            sm100::mbar_init(q_free + s, 1);
+            sm100::mbar_init(o_full + s, 1);
+            sm100::mbar_init(o_free + s, 128);
+        }
+        for (int s = 0; s < NSB; ++s) {
             sm100::mbar_init(s_full + s, 1);
             sm100::mbar_init(p_full + s, 128);
         }
-        sm100::mbar_init(o_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            sm100::mbar_init(k_full + s, 1);
+            sm100::mbar_init(k_ready + s, 128);
+            sm100::mbar_init(v_full + s, 1);
+            sm100::mbar_init(release + s, 1);
+        }
         sm100::mbar_init(o_upd, 1);
         sm100::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -208,12 +549,17 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     const int ptid = threadIdx.x - 32 * FWD_PREP_WARP0;   // 0..127 inside the prep group
     const bool is_prep = warp >= FWD_PREP_WARP0 && warp < FWD_PREP_WARP0 + 4;
+    RotThread rot;
     if (is_prep && a.use_rope) {
         if (ptid < D / 2) sTh[ptid] = exp2(-2.0 * (double)ptid / (double)D * a.log2_base);
         sm100::named_bar_sync(FWD_PREP_BAR, 128);
-        for (int e = ptid; e < (D / 2) * 32; e += 128) {
-            int t = e / 32, l = e % 32;
-            sW[e] = rope_cs((double)l * sTh[t]);
+        constexpr int CPR = D / 8, RS = 128 / CPR;
+        const int c = ptid % CPR, r0 = ptid / CPR;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const double th = sTh[4 * c + q];
+            const float2 w0 = rope_cs((double)r0 * th), stp = rope_cs((double)RS * th);
+            rot.w0c[q] = w0.x; rot.w0s[q] = w0.y; rot.stc[q] = stp.x; rot.sts[q] = stp.y;
         }
     }
     sm100::tc_fence_before();
@@ -221,60 +567,71 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    FwdSched S;
+    S.init(a, NS, blockIdx.x, gridDim.x);
+    FwdStep st;
+
     if (warp == FWD_TMA_WARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int last_n[NST];
-            for (int s = 0; s < NST; ++s) last_n[s] = -1;
-            sm100::mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
-            for (int hh = 0; hh < D / 64; ++hh)
-                sm100::tma_load_4d(sQ + hh * C::HALF_BYTES, &tm_q, q_full, hh * 64, h, i0, b);
-            for (int t = 0; t < T; ++t) {
-                const int st = t % NST, n = t / NST;
-                if (n > 0 && !sm100::mbar_wait(kv_empty + st, (n - 1) & 1, abort_flag)) break;
-                const int j0 = fwd_tile_j0(tr, t);
-                sm100::mbar_arrive_expect_tx(k_full + st, C::TILE_BYTES);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    sm100::tma_load_4d(sK + st * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_k, k_full + st,
-                                       hh * 64, kvh, j0, b);
-                sm100::mbar_arrive_expect_tx(v_full + st, C::TILE_BYTES);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    sm100::tma_load_4d(sV + st * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_v, v_full + st,
-                                       hh * 64, kvh, j0, b);
-                last_n[st] = n;
+            int last_par[NS];
+            for (int s = 0; s < NS; ++s) last_par[s] = -1;
+            int nq = 0;
+            while (S.next_step(st)) {
+                if (st.first) {
+                    const int qs = st.k & 1;
+                    if (st.k >= 2 && !sm100::mbar_wait(q_free + qs, ((st.k - 2) >> 1) & 1, abort_flag)) break;
+                    sm100::mbar_arrive_expect_tx(q_full + qs, C::TILE_BYTES);
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        sm100::tma_load_4d(sQ + qs * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_q, q_full + qs,
+                                           hh * 64, st.h, st.i0, st.b);
+                    nq = st.k + 1;
+                }
+                if (st.is_new) {
+                    if (st.need_release && !sm100::mbar_wait(release + st.slot, st.par ^ 1, abort_flag)) break;
+                    sm100::mbar_arrive_expect_tx(k_full + st.slot, C::TILE_BYTES);
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        sm100::tma_load_4d(sK + st.slot * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_k,
+                                           k_full + st.slot, hh * 64, st.kvh, st.j0, st.b);
+                    sm100::mbar_arrive_expect_tx(v_full + st.slot, C::TILE_BYTES);
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        sm100::tma_load_4d(sV + st.slot * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_v,
+                                           v_full + st.slot, hh * 64, st.kvh, st.j0, st.b);
+                    last_par[st.slot] = st.par;
+                }
             }
             // every issued copy must have landed before the CTA may exit
-            mbar_wait_drain(q_full, 0);
-            for (int s = 0; s < NST; ++s)
-                if (last_n[s] >= 0) {
-                    mbar_wait_drain(k_full + s, last_n[s] & 1);
-                    mbar_wait_drain(v_full + s, last_n[s] & 1);
+            for (int kq = max(0, nq - 2); kq < nq; ++kq) mbar_wait_drain(q_full + (kq & 1), (kq >> 1) & 1);
+            for (int s = 0; s < NS; ++s)
+                if (last_par[s] >= 0) {
+                    mbar_wait_drain(k_full + s, last_par[s]);
+                    mbar_wait_drain(v_full + s, last_par[s]);
                 }
         }
     } else if (is_prep) {
         // ------------------------------------------------------------ RoPE prep
-        const int w = ptid / 32, l = ptid % 32;
-        auto make_bases = [&](int buf, int pos0) {
-            if (!a.use_rope) return;
-            for (int e = ptid; e < 4 * (D / 2); e += 128) {
-                int ww = e / (D / 2), t = e % (D / 2);
-                sE[buf * 4 * (D / 2) + e] = rope_cs((double)(pos0 + 32 * ww) * sTh[t]);
-            }
+        int ebuf = 0;
+        auto make_bases = [&](int pos0) {
+            ebuf ^= 1;
+            if (a.use_rope && ptid < D / 2) sE[ebuf * (D / 2) + ptid] = rope_cs((double)pos0 * sTh[ptid]);
         };
-        make_bases(0, i0);
-        bool ok = sm100::mbar_wait(q_full, 0, abort_flag);
-        if (!named_bar_or(FWD_PREP_BAR, 128, !ok || *abort_flag)) {
-            if (a.use_rope) rope_rotate_tile<D>(sQ, sW, sE, w, l);
-            sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(q_ready);
-            for (int t = 0; t < T; ++t) {
-                const int st = t % NST, n = t / NST, buf = (t + 1) & 1;
-                make_bases(buf, fwd_tile_j0(tr, t));
-                ok = sm100::mbar_wait(k_full + st, n & 1, abort_flag);
+        while (S.next_step(st)) {
+            if (st.first) {
+                const int qs = st.k & 1;
+                make_bases(st.i0);
+                const bool ok = sm100::mbar_wait(q_full + qs, (st.k >> 1) & 1, abort_flag);
                 if (named_bar_or(FWD_PREP_BAR, 128, !ok || *abort_flag)) break;
-                if (a.use_rope) rope_rotate_tile<D>(sK + st * C::TILE_BYTES, sW, sE + buf * 4 * (D / 2), w, l);
+                if (a.use_rope) rope_rotate_tile<D>(sQ + qs * C::TILE_BYTES, sE + ebuf * (D / 2), rot, ptid);
                 sm100::fence_proxy_async_smem();
-                sm100::mbar_arrive(k_ready + st);
+                sm100::mbar_arrive(q_ready + qs);
+            }
+            if (st.is_new) {
+                make_bases(st.j0);
+                const bool ok = sm100::mbar_wait(k_full + st.slot, st.par, abort_flag);
+                if (named_bar_or(FWD_PREP_BAR, 128, !ok || *abort_flag)) break;
+                if (a.use_rope) rope_rotate_tile<D>(sK + st.slot * C::TILE_BYTES, sE + ebuf * (D / 2), rot, ptid);
+                sm100::fence_proxy_async_smem();
+                sm100::mbar_arrive(k_ready + st.slot);
             }
         }
     } else if (warp == FWD_MMA_WARP) {
@@ -282,183 +639,154 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (lane == 0) {
             constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t IDESC_PV = sm100::idesc_bf16_f32(128, D, 0, 1);
-            const uint32_t qa = sm100::smem_u32(sQ);
-            auto issue_pv = [&](int u) -> bool {
-                const int st = u % NST, bb = u & 1;
-                if (!sm100::mbar_wait(p_full + bb, (u >> 1) & 1, abort_flag)) return false;
-                if (!sm100::mbar_wait(v_full + st, (u / NST) & 1, abort_flag)) return false;
+            // descriptor words: high half fixed per operand kind, low half = start address >> 4 (+ LBO)
+            const uint64_t dq0 = sm100::sdesc_sw128(sm100::smem_u32(sQ), 16, 1024);
+            const uint64_t dk0 = sm100::sdesc_sw128(sm100::smem_u32(sK), 16, 1024);
+            const uint64_t dv0 = sm100::sdesc_sw128(sm100::smem_u32(sV), C::HALF_BYTES, 1024);
+            const uint32_t hi_k = (uint32_t)(dk0 >> 32), hi_v = (uint32_t)(dv0 >> 32);
+            const uint32_t lo_q = (uint32_t)dq0, lo_k = (uint32_t)dk0, lo_v = (uint32_t)dv0;
+            constexpr uint32_t TILE16 = C::TILE_BYTES >> 4, HALF16 = C::HALF_BYTES >> 4;
+            auto mk = [](uint32_t hi, uint32_t lo) { return ((uint64_t)hi << 32) | lo; };
+            auto issue_pv = [&](const FwdStep &p) -> bool {
+                const int sb = p.step % NSB, ob = p.k & 1;
+                if (!sm100::mbar_wait(p_full + sb, (p.step / NSB) & 1, abort_flag)) return false;
+                if (p.is_new && !sm100::mbar_wait(v_full + p.slot, p.par, abort_flag)) return false;
+                if (p.first && p.k >= 2 && !sm100::mbar_wait(o_free + ob, ((p.k - 2) >> 1) & 1, abort_flag))
+                    return false;
                 sm100::tc_fence_after();
-                const uint32_t va = sm100::smem_u32(sV + st * C::TILE_BYTES);
+                const uint32_t lv = lo_v + (uint32_t)p.slot * TILE16;
+                const uint32_t d_o = tmem + C::COL_O + ob * D, a_p = tmem + sb * 128;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t bd = sm100::sdesc_sw128(va + ks * 2048, C::HALF_BYTES, 1024);
-                    sm100::umma_ts(tmem + C::COL_O, tmem + bb * 128 + ks * 8, bd, IDESC_PV,
-                                   (u > 0 || ks > 0) ? 1u : 0u);
-                }
-                sm100::umma_commit(kv_empty + st);
+                for (int ks = 0; ks < 8; ++ks)
+                    sm100::umma_ts(d_o, a_p + ks * 8, mk(hi_v, lv + ks * (2048 >> 4)), IDESC_PV,
+                                   (!p.first || ks > 0) ? 1u : 0u);
+                if (p.last_use) sm100::umma_commit(release + p.slot);
                 if (MODE == SWAT_MODE_SOFTMAX_) sm100::umma_commit(o_upd);
+                if (p.last) sm100::umma_commit(o_full + ob);
                 return true;
             };
-            bool ok = sm100::mbar_wait(q_ready, 0, abort_flag);
-            for (int t = 0; ok && t < T; ++t) {
-                const int st = t % NST, n = t / NST, bb = t & 1;
-                if (!sm100::mbar_wait(k_ready + st, n & 1, abort_flag)) { ok = false; break; }
+            // S runs up to NSB-1 steps ahead of P.V: the S buffer of step s is
+            // reused by step s + NSB, whose S is issued after PV(s).
+            FwdStep pend0, pend1;
+            int npend = 0;
+            bool ok = true;
+            while (ok && S.next_step(st)) {
+                const int qs = st.k & 1, sb = st.step % NSB;
+                if (st.first && !sm100::mbar_wait(q_ready + qs, (st.k >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (st.is_new && !sm100::mbar_wait(k_ready + st.slot, st.par, abort_flag)) { ok = false; break; }
                 sm100::tc_fence_after();
-                const uint32_t ka = sm100::smem_u32(sK + st * C::TILE_BYTES);
+                const uint32_t lq = lo_q + (uint32_t)qs * TILE16, lk = lo_k + (uint32_t)st.slot * TILE16;
+                const uint32_t d_s = tmem + sb * 128;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
-                    const uint64_t ad = sm100::sdesc_sw128(qa + off, 16, 1024);
-                    const uint64_t bd = sm100::sdesc_sw128(ka + off, 16, 1024);
-                    sm100::umma_ss(tmem + bb * 128, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
+                    const uint32_t off = (ks / 4) * HALF16 + (ks % 4) * 2;
+                    sm100::umma_ss(d_s, mk(hi_k, lq + off), mk(hi_k, lk + off), IDESC_S, ks > 0 ? 1u : 0u);
                 }
-                sm100::umma_commit(s_full + bb);
-                if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+                sm100::umma_commit(s_full + sb);
+                if (st.last) sm100::umma_commit(q_free + qs);
+                if (npend == NSB - 1) {
+                    if (!issue_pv(pend0)) { ok = false; break; }
+                    pend0 = pend1;
+                    --npend;
+                }
+                if (npend == 0) pend0 = st; else pend1 = st;
+                ++npend;
             }
-            if (ok) ok = issue_pv(T - 1);
-            if (ok) sm100::umma_commit(o_full);
+            if (ok && npend > 0) ok = issue_pv(pend0);
+            if (ok && npend > 1) ok = issue_pv(pend1);
             sm100::umma_commit(drain);
             mbar_wait_drain(drain, 0);   // nothing of ours is in flight past this point
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------ activation
-        const int r = 32 * warp + lane;                  // query row inside the tile (= TMEM lane)
-        const int i = i0 + r;
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-        const float slope = a.slopes ? a.slopes[h] : 0.f;
+    } else if (warp >= FWD_ACT_WARP0) {
+        // ------------------------------------------------------------ activation + epilogue
+        const int aw = (warp - FWD_ACT_WARP0) / 4;       // activation warpgroup
+        const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
+        const int r = 32 * (warp % 4) + lane;            // query row inside the tile (= TMEM lane)
         float m_used = -INFINITY, l_sum = 0.f;           // softmax state (log2 domain)
-        bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int bb = t & 1;
-            ok = sm100::mbar_wait(s_full + bb, (t >> 1) & 1, abort_flag);
-            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+        const float LOG2E = 1.4426950408889634f;
+        while (S.next_step(st)) {
+            const int sb = st.step % NSB;
+            if (RL::ACT_WG == 2 && (st.step & 1) != aw) continue;   // the other warpgroup's tile
+            const int i = st.i0 + r;
+            const float slope = a.slopes ? __ldg(a.slopes + st.h) : 0.f;
+            if (st.first) { m_used = -INFINITY; l_sum = 0.f; }
+            bool ok = sm100::mbar_wait(s_full + sb, (st.step / NSB) & 1, abort_flag);
+            if (__any_sync(0xffffffffu, !ok)) break;
             sm100::tc_fence_after();
-            const int j0 = fwd_tile_j0(tr, t);
-            const bool need_mask = !(j0 + 127 <= i0 && (i0 + 127 - j0 < a.window || j0 + 127 < a.n_sink));
-            const int rd = i - j0;                       // i - j at column 0
-            const uint32_t s_addr = tmem + lane_base + bb * 128;
+            const int j0 = st.j0, i0 = st.i0;
+            const bool masked = !(j0 + 127 <= i0 && (i0 + 127 - j0 < a.window || j0 + 127 < a.n_sink));
+            const int rd = i - j0;
+            const uint32_t s_addr = tmem + lane_base + sb * 128;
             if (MODE == SWAT_MODE_SIGMOID_) {
-                // sigma(x) = 0.5 + 0.5 tanh(x / 2), x = acc/sqrt(d) + slope (i - j)
-                const float hs = 0.5f * a.scale, hsl = 0.5f * slope, hb0 = hsl * (float)rd;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    uint32_t v[32];
-                    sm100::tmem_ld32(s_addr + 32 * k, v);
-                    sm100::tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c0 = 32 * k + 2 * e, c1 = c0 + 1;
-                        float x0 = fmaf(__uint_as_float(v[2 * e]), hs, fmaf(-hsl, (float)c0, hb0));
-                        float x1 = fmaf(__uint_as_float(v[2 * e + 1]), hs, fmaf(-hsl, (float)c1, hb0));
-                        float p0 = fmaf(0.5f, sm100::tanh_approx(x0), 0.5f);
-                        float p1 = fmaf(0.5f, sm100::tanh_approx(x1), 0.5f);
-                        if (need_mask) {
-                            const int d0 = rd - c0, d1 = rd - c1;
-                            if (!(d0 >= 0 && (d0 < a.window || j0 + c0 < a.n_sink))) p0 = 0.f;
-                            if (!(d1 >= 0 && (d1 < a.window || j0 + c1 < a.n_sink))) p1 = 0.f;
-                        }
-                        pk[e] = sm100::pack_bf16x2(p0, p1);
-                    }
-                    sm100::tmem_st16(s_addr + 16 * k, pk);
-                }
+                const float hs = 0.5f * a.scale, hsl = 0.5f * slope;
+                const int rd_w0 = st.i0 + 32 * (warp % 4) - j0;   // first row of this warp
+                if (masked) act_sigmoid_tile<true>(s_addr, hs, hsl, rd, rd_w0, j0, a.window, a.n_sink);
+                else act_sigmoid_tile<false>(s_addr, hs, hsl, rd, rd_w0, j0, a.window, a.n_sink);
             } else {
-                // softmax in the log2 domain: x2 = log2(e) * s
-                const float LOG2E = 1.4426950408889634f;
-                const float sc2 = a.scale * LOG2E, sl2 = slope * LOG2E, b2 = sl2 * (float)rd;
-                float mx = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    uint32_t v[32];
-                    sm100::tmem_ld32(s_addr + 32 * k, v);
-                    sm100::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = 32 * k + e;
-                        float x = fmaf(__uint_as_float(v[e]), sc2, fmaf(-sl2, (float)c, b2));
-                        if (need_mask) {
-                            const int dd = rd - c;
-                            if (!(dd >= 0 && (dd < a.window || j0 + c < a.n_sink))) x = -INFINITY;
-                        }
-                        mx = fmaxf(mx, x);
-                    }
-                }
+                const float sc2 = a.scale * LOG2E, sl2 = slope * LOG2E;
+                const float mx = masked ? act_softmax_max<true>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink)
+                                        : act_softmax_max<false>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink);
                 // keep a stale maximum while the new one exceeds it by at most 8
                 // (weights stay <= 2^8); otherwise rescale this row of O and l
                 const bool need = mx > m_used + 8.0f;
                 const bool need_o = need && m_used != -INFINITY;
                 if (__any_sync(0xffffffffu, need_o)) {
-                    if (!sm100::mbar_wait(o_upd, (t - 1) & 1, abort_flag)) ok = false;
-                    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                    ok = sm100::mbar_wait(o_upd, (st.step - 1) & 1, abort_flag);
+                    if (__any_sync(0xffffffffu, !ok)) break;
                     sm100::tc_fence_after();
                     const float f = need_o ? sm100::ex2_approx(m_used - mx) : 1.f;
+                    const uint32_t o_addr = tmem + lane_base + C::COL_O + (st.k & 1) * D;
 #pragma unroll
-                    for (int k = 0; k < D / 32; ++k) {
+                    for (int kk = 0; kk < D / 32; ++kk) {
                         uint32_t v[32];
-                        sm100::tmem_ld32(tmem + lane_base + C::COL_O + 32 * k, v);
-                        sm100::tmem_wait_ld();
+                        sm100::tmem_ld32(o_addr + 32 * kk, v);
+                        sm100::tmem_wait_ld_dep(v);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-                        sm100::tmem_st32(tmem + lane_base + C::COL_O + 32 * k, v);
+                        sm100::tmem_st32(o_addr + 32 * kk, v);
                     }
                     if (need_o) l_sum *= f;
                 }
                 if (need) m_used = mx;
-                float lsum = 0.f;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    uint32_t v[32];
-                    sm100::tmem_ld32(s_addr + 32 * k, v);
-                    sm100::tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c0 = 32 * k + 2 * e, c1 = c0 + 1;
-                        float x0 = fmaf(__uint_as_float(v[2 * e]), sc2, fmaf(-sl2, (float)c0, b2));
-                        float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sc2, fmaf(-sl2, (float)c1, b2));
-                        float p0 = (m_used == -INFINITY) ? 0.f : sm100::ex2_approx(x0 - m_used);
-                        float p1 = (m_used == -INFINITY) ? 0.f : sm100::ex2_approx(x1 - m_used);
-                        if (need_mask) {
-                            const int d0 = rd - c0, d1 = rd - c1;
-                            if (!(d0 >= 0 && (d0 < a.window || j0 + c0 < a.n_sink))) p0 = 0.f;
-                            if (!(d1 >= 0 && (d1 < a.window || j0 + c1 < a.n_sink))) p1 = 0.f;
-                        }
-                        lsum += p0 + p1;
-                        pk[e] = sm100::pack_bf16x2(p0, p1);
-                    }
-                    sm100::tmem_st16(s_addr + 16 * k, pk);
-                }
-                l_sum += lsum;
+                l_sum += masked ? act_softmax_p<true>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink, m_used)
+                                : act_softmax_p<false>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink, m_used);
             }
             sm100::tmem_wait_st();
             sm100::tc_fence_before();
-            sm100::mbar_arrive(p_full + bb);
-        }
-        // ---- epilogue: O (TMEM) -> registers -> global, one row per thread
-        if (ok) ok = sm100::mbar_wait(o_full, 0, abort_flag);
-        if (!__any_sync(0xffffffffu, !ok)) {
-            sm100::tc_fence_after();
-            float inv = 1.f;
-            if (MODE == SWAT_MODE_SOFTMAX_) inv = 1.f / l_sum;
-            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.N + i) * a.H + h) * D;
+            sm100::mbar_arrive(p_full + sb);
+            if (st.last) {
+                // ---- epilogue of the item: O (TMEM) -> registers -> global, one row per thread
+                const int ob = st.k & 1;
+                ok = sm100::mbar_wait(o_full + ob, (st.k >> 1) & 1, abort_flag);
+                if (__any_sync(0xffffffffu, !ok)) break;
+                sm100::tc_fence_after();
+                const float inv = (MODE == SWAT_MODE_SOFTMAX_) ? 1.f / l_sum : 1.f;
+                __nv_bfloat16 *orow =
+                    reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)st.b * a.N + i) * a.H + st.h) * D;
+                const uint32_t o_addr = tmem + lane_base + C::COL_O + ob * D;
 #pragma unroll
-            for (int k = 0; k < D / 32; ++k) {
-                uint32_t v[32];
-                sm100::tmem_ld32(tmem + lane_base + C::COL_O + 32 * k, v);
-                sm100::tmem_wait_ld();
-                if (i < a.N) {
-                    uint32_t pk[16];
+                for (int kk = 0; kk < D / 32; ++kk) {
+                    uint32_t v[32];
+                    sm100::tmem_ld32(o_addr + 32 * kk, v);
+                    sm100::tmem_wait_ld_dep(v);
+                    if (i < a.N) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = sm100::pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * k);
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = sm100::pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
+                                                       __uint_as_float(v[2 * e + 1]) * inv);
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * kk);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
                 }
+                if (MODE == SWAT_MODE_SOFTMAX_ && i < a.N)
+                    a.lse[((size_t)st.b * a.H + st.h) * a.N + i] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
+                sm100::tc_fence_before();
+                sm100::mbar_arrive(o_free + ob);
             }
-            if (MODE == SWAT_MODE_SOFTMAX_ && i < a.N)
-                a.lse[((size_t)b * a.H + h) * a.N + i] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
         }
     }
 
@@ -503,6 +831,14 @@ inline bool make_tmap_bshd(CUtensorMap *m, const void *ptr, int B, int N, int Hx
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+inline int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
 template <int D, int MODE>
 inline int launch_fwd_tc_t(const FwdArgs &a, cudaStream_t stream)
 {
@@ -513,8 +849,10 @@ inline int launch_fwd_tc_t(const FwdArgs &a, cudaStream_t stream)
         return -1;
     auto kern = swat_fwd_tc_kernel<D, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return -1;
-    dim3 grid((a.N + 127) / 128, a.H, a.B);
-    kern<<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, a);
+    const long long items = (long long)a.B * a.H * ((a.N + 127) / 128);
+    if (items >= (1LL << 31)) return -1;   // the schedule decodes item indices in 32 bits
+    const int grid = (int)std::min<long long>(items, (long long)num_sms());
+    kern<<<grid, FwdRoles<MODE>::THREADS, C::SMEM, stream>>>(tq, tk, tv, a);
     return 1;
 }
 
