@@ -125,3 +125,23 @@ def test_decode_after_fill_equals_forward_row():
     for p in range(P, N):
         o = rc.step(q[:, p], k[:, p], v[:, p], np.full(B, p), mode=1)
         np.testing.assert_allclose(o, o_ref[:, p], atol=1e-12)
+
+
+@pytest.mark.parametrize("mode,Hkv,w,s", [(0, 2, 9, 0), (1, 1, 7, 3), (1, 4, 100, 2), (0, 2, 5, 4)])
+def test_bwd_c_oracle_equals_dense_numpy_bwd(mode, Hkv, w, s):
+    """Two backward derivations written independently (per-row C loops vs
+    dense numpy matrices) agree to rounding."""
+    from oracle import ref_numpy
+    q, k, v, do = [t.numpy().astype(np.float32) for t in
+                   inputs.qkv(2, 37, 4, Hkv, 8, seed=11, dtype=torch.float32, with_dout=True)]
+    sl = inputs.balanced_alibi_slopes(4).numpy()
+    kw = dict(window=w, n_sink=s, mode=mode, slopes=sl, rope_base=1e4)
+    for a, b in zip(oracle.swat_bwd(q, k, v, do, **kw), ref_numpy.swat_bwd(q, k, v, do, **kw)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-11)
+
+
+def test_round_bf16_helper_matches_torch_cast():
+    from tests.helpers import round_bf16
+    x = np.random.default_rng(0).standard_normal(50000).astype(np.float32) * 7
+    x[:4] = [0.0, -0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8]   # exact ties
+    assert np.array_equal(round_bf16(x), torch.tensor(x).bfloat16().double().numpy())
