@@ -12,6 +12,7 @@
 #include "bwd_simt.cuh"
 #include "decode.cuh"
 #include "fwd_tc.cuh"
+#include "bwd_tc.cuh"
 #include "decode_fast.cuh"
 
 namespace {
@@ -142,13 +143,10 @@ int swat_attn_bwd(const void *q, const void *k, const void *v, const void *o, co
     a.mode = mode; a.use_rope = rope_base > 0.f; a.log2_base = log2_base_of(rope_base);
     a.scale = (float)(1.0 / sqrt((double)d));
     int n = 0;
-    if (mode == SWAT_MODE_SOFTMAX) {
+    if (mode == SWAT_MODE_SOFTMAX && dtype == SWAT_F32) {   // (the bf16 path computes D_i itself)
         long long rows = (long long)B * N * H;
         int threads = 256, rpb = threads / 32;
-        if (dtype == SWAT_BF16)
-            swat::swat_bwd_dot_do_o_kernel<__nv_bfloat16><<<(unsigned)((rows + rpb - 1) / rpb), threads, 0, S(stream)>>>(a);
-        else
-            swat::swat_bwd_dot_do_o_kernel<float><<<(unsigned)((rows + rpb - 1) / rpb), threads, 0, S(stream)>>>(a);
+        swat::swat_bwd_dot_do_o_kernel<float><<<(unsigned)((rows + rpb - 1) / rpb), threads, 0, S(stream)>>>(a);
         ++n;
     }
     if (dtype == SWAT_BF16) {

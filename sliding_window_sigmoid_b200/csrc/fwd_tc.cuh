@@ -868,26 +868,4 @@ inline int launch_fwd_tc(const TcFwdArgs &a, cudaStream_t stream)
     return -1;
 }
 
-// ---------------------------------------------------------------------------
-// bf16 backward (CUDA-core kernels for now)
-// ---------------------------------------------------------------------------
-inline size_t tc_bwd_extra_workspace(int B, int H, int Hkv, int N, int d)
-{
-    (void)B; (void)H; (void)Hkv; (void)N; (void)d;
-    return 0;
-}
-
-inline int launch_bwd_tc(const BwdArgs &a, void *extra_ws, cudaStream_t stream)
-{
-    (void)extra_ws;
-    size_t smem_q = simt_bwd_dq_smem_bytes(), smem_k = simt_bwd_dkdv_smem_bytes();
-    cudaFuncSetAttribute(swat_bwd_dq_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q);
-    cudaFuncSetAttribute(swat_bwd_dkdv_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k);
-    dim3 gq((a.N + SIMT_BQ - 1) / SIMT_BQ, a.H, a.B);
-    dim3 gk((a.N + SIMT_BK - 1) / SIMT_BK, a.Hkv, a.B);
-    swat_bwd_dq_simt_kernel<__nv_bfloat16><<<gq, SIMT_THREADS, smem_q, stream>>>(a);
-    swat_bwd_dkdv_simt_kernel<__nv_bfloat16><<<gk, SIMT_THREADS, smem_k, stream>>>(a);
-    return 2;
-}
-
 }  // namespace swat
