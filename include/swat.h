@@ -64,7 +64,8 @@ typedef enum {
     SWAT_ERR_INVALID_ARG = -1,
     SWAT_ERR_UNSUPPORTED = -2,
     SWAT_ERR_CUDA = -3,
-    SWAT_ERR_TIMEOUT = -4
+    SWAT_ERR_TIMEOUT = -4,
+    SWAT_ERR_SCRATCH_LIMIT = -5
 } swat_status_t;
 
 typedef enum { SWAT_MODE_SIGMOID = 0, SWAT_MODE_SOFTMAX = 1 } swat_mode_t;
@@ -136,6 +137,44 @@ SWAT_API int swa_decode_step(const void *q, const void *k_new, const void *v_new
 
 /* Bytes of device workspace swa_decode_step needs. */
 SWAT_API size_t swa_decode_workspace_bytes(int B, int H, int Hkv, int d, int window);
+
+/* Size of the library's own decode scratch buffer (16 MiB of device memory
+ * per device, reserved when the library's device code is loaded). A decode
+ * step fits iff swa_decode_workspace_bytes(B, H, Hkv, d, window) is at most
+ * this: e.g. 64 sequences x 32 query heads, d 128, window 4096 need 8.1 MiB. */
+#define SWA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* swa_decode_step without a workspace argument: the same decode step, same
+ * kernels and same results, with the split partials kept in the library's
+ * own static device buffer (SWA_DECODE_NOALLOC_SCRATCH_BYTES). It allocates
+ * no device memory, ever. This entry point has no counterpart in the pages:
+ * it exists for callers that cannot hand over a workspace, such as a C host
+ * with no device allocator of its own, or a serving loop that must not call
+ * cudaMalloc/cudaFree between steps because those calls synchronise the
+ * device and stall its other streams.
+ *
+ * Arguments, layouts, ownership and the key set are those of swa_decode_step
+ * (minus `workspace`).
+ *
+ * - The first call on each device does a one-time set-up: with that device
+ *   current it looks up the buffer's device address. Make that first call
+ *   before any stream capture begins. Call with the device that owns the
+ *   buffers and `stream` current.
+ * - Nothing in the buffer has to start at zero: each step writes every
+ *   partial before it reads it.
+ * - There is ONE buffer per device: two calls whose work can overlap on the
+ *   device (different streams without ordering between them, or concurrent
+ *   host threads) race on it and corrupt each other's results. Order such
+ *   calls on one stream or with events.
+ * - Returns SWAT_ERR_SCRATCH_LIMIT, before any launch, when the step needs
+ *   more than SWA_DECODE_NOALLOC_SCRATCH_BYTES (use swa_decode_step with a
+ *   workspace for such shapes); SWAT_ERR_CUDA if the set-up lookup fails;
+ *   otherwise whatever swa_decode_step returns. */
+SWAT_API int swa_decode_step_noalloc(const void *q, const void *k_new, const void *v_new,
+                    void *k_cache, void *v_cache, void *k_sink, void *v_sink,
+                    const long long *pos, void *o,
+                    int B, int H, int Hkv, int d, int window, int n_sink, int mode,
+                    const float *slopes, float rope_base, int dtype, void *stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 SWAT_API const char *swat_status_string(int status);

@@ -22,10 +22,12 @@ BF16 = 0
 F32 = 1
 
 _STATUS = {0: "SWAT_OK", -1: "SWAT_ERR_INVALID_ARG", -2: "SWAT_ERR_UNSUPPORTED",
-           -3: "SWAT_ERR_CUDA", -4: "SWAT_ERR_TIMEOUT"}
+           -3: "SWAT_ERR_CUDA", -4: "SWAT_ERR_TIMEOUT", -5: "SWAT_ERR_SCRATCH_LIMIT"}
+SCRATCH_LIMIT = -5
+NOALLOC_SCRATCH_BYTES = 16 << 20   # SWA_DECODE_NOALLOC_SCRATCH_BYTES
 
 EXPORTED = ["swat_attn_fwd", "swat_attn_bwd_workspace_bytes", "swat_attn_bwd", "swa_cache_fill",
-            "swa_decode_step", "swa_decode_workspace_bytes", "swat_status_string",
+            "swa_decode_step", "swa_decode_workspace_bytes", "swa_decode_step_noalloc", "swat_status_string",
             "swat_get_device_status", "swat_launch_count"]
 
 
@@ -58,6 +60,8 @@ def lib() -> ctypes.CDLL:
     L.swa_cache_fill.restype = I
     L.swa_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, F, I, P]
     L.swa_decode_step.restype = I
+    L.swa_decode_step_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, F, I, P]
+    L.swa_decode_step_noalloc.restype = I
     L.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     L.swa_decode_workspace_bytes.restype = SZ
     L.swat_status_string.argtypes = [I]
@@ -208,6 +212,23 @@ class RingCache:
                                    self.Hkv, self.d, self.window, self.n_sink, self.mode,
                                    _ptr(self.slopes), self.rope_base, self._code, _stream(stream))
         _check("swa_decode_step", st)
+        return out
+
+    def step_noalloc(self, q, k_new, v_new, pos, out=None, stream=None):
+        """The same step through swa_decode_step_noalloc: the library's own
+        static scratch buffer instead of this object's workspace (calls that
+        can overlap on the device must not use it concurrently)."""
+        _need(q, "q", (self.B, self.H, self.d), self.dtype, self.device)
+        _need(k_new, "k_new", (self.B, self.Hkv, self.d), self.dtype, self.device)
+        _need(v_new, "v_new", (self.B, self.Hkv, self.d), self.dtype, self.device)
+        _need(pos, "pos", (self.B,), torch.int64, self.device)
+        out = torch.empty_like(q) if out is None else out
+        st = lib().swa_decode_step_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(self.k_cache),
+                                           _ptr(self.v_cache), _ptr(self.k_sink), _ptr(self.v_sink),
+                                           _ptr(pos), _ptr(out), self.B, self.H, self.Hkv, self.d,
+                                           self.window, self.n_sink, self.mode, _ptr(self.slopes),
+                                           self.rope_base, self._code, _stream(stream))
+        _check("swa_decode_step_noalloc", st)
         return out
 
 

@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdio.h>
 #include <atomic>
+#include <mutex>
 
 #include "swat.h"
 #include "common.cuh"
@@ -59,6 +60,7 @@ const char *swat_status_string(int status)
         case SWAT_ERR_UNSUPPORTED: return "SWAT_ERR_UNSUPPORTED";
         case SWAT_ERR_CUDA: return "SWAT_ERR_CUDA";
         case SWAT_ERR_TIMEOUT: return "SWAT_ERR_TIMEOUT";
+        case SWAT_ERR_SCRATCH_LIMIT: return "SWAT_ERR_SCRATCH_LIMIT";
         default: return "SWAT_ERR_UNKNOWN";
     }
 }
@@ -248,3 +250,61 @@ int swa_decode_step(const void *q, const void *k_new, const void *v_new,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode step with library-owned scratch (no workspace argument, no allocation)
+//
+// The split partials that swa_decode_step keeps in the caller's workspace live
+// here in one file-scope device buffer instead. Its device address is looked
+// up once per device (cudaGetSymbolAddress with that device current) and then
+// reused; the decode kernels themselves are the ones swa_decode_step runs.
+// Every partial is written by the attention pass before the combine pass reads
+// it, so the buffer's contents never need to start at zero.
+static __device__ __align__(256) unsigned char g_decode_scratch[SWA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::atomic<void *> g_decode_scratch_ptr[kMaxScratchDevices];
+std::mutex g_decode_scratch_mu;
+
+// Device address of g_decode_scratch on the current device (set-up on first use).
+int decode_scratch_current_device(void **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SWAT_ERR_CUDA; }
+    if (dev < 0 || dev >= kMaxScratchDevices) return SWAT_ERR_UNSUPPORTED;
+    void *p = g_decode_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_decode_scratch_mu);
+        p = g_decode_scratch_ptr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+            if (e != cudaSuccess || !p) { cudaGetLastError(); return SWAT_ERR_CUDA; }
+            g_decode_scratch_ptr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return SWAT_OK;
+}
+
+}  // namespace
+
+extern "C" int swa_decode_step_noalloc(const void *q, const void *k_new, const void *v_new,
+                                       void *k_cache, void *v_cache, void *k_sink, void *v_sink,
+                                       const long long *pos, void *o,
+                                       int B, int H, int Hkv, int d, int window, int n_sink,
+                                       int mode, const float *slopes, float rope_base, int dtype,
+                                       void *stream)
+{
+    int st = check_attn_shapes(B, H, Hkv, 1, d, window, n_sink, mode, dtype);
+    if (st != SWAT_OK) return st;
+    const size_t need = swa_decode_workspace_bytes(B, H, Hkv, d, window);
+    if (need == 0) return SWAT_ERR_INVALID_ARG;
+    if (need > (size_t)SWA_DECODE_NOALLOC_SCRATCH_BYTES) return SWAT_ERR_SCRATCH_LIMIT;
+    void *scratch = nullptr;
+    st = decode_scratch_current_device(&scratch);
+    if (st != SWAT_OK) return st;
+    return swa_decode_step(q, k_new, v_new, k_cache, v_cache, k_sink, v_sink, pos, o, scratch,
+                           B, H, Hkv, d, window, n_sink, mode, slopes, rope_base, dtype, stream);
+}
