@@ -222,7 +222,7 @@ def run_swat(args):
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local if world > 1 else 0)
     wl = inputs.SWAT_340M
-    B, H, Hkv, N, d, w = wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.window
+    B, H, Hkv, N, d, w = args.batch or wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.window
     kw = dict(window=w, n_sink=0, mode=binding.MODE_SIGMOID, slopes=wl.slope_tensor(),
               rope_base=wl.rope_base)
     q, k, v, do = [t.to(dev) for t in inputs.qkv(B, N, H, Hkv, d, seed=100 * rank, scale=wl.scale,
@@ -375,7 +375,7 @@ def bench_decode(args, dev, world, rank, peaks, peak_src):
     out = {}
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     for wl in (inputs.DECODE_SIGMOID, inputs.DECODE_SOFTMAX):
-        B, H, Hkv, d, w, s = wl.B, wl.H, wl.Hkv, wl.d, wl.window, wl.n_sink
+        B, H, Hkv, d, w, s = args.decode_batch or wl.B, wl.H, wl.Hkv, wl.d, wl.window, wl.n_sink
         cache = binding.RingCache(B, H, Hkv, d, w, s, mode=wl.mode, slopes=wl.slope_tensor(),
                                   rope_base=wl.rope_base, device=dev)
         g = torch.Generator(device=dev)
@@ -409,7 +409,7 @@ def bench_decode(args, dev, world, rank, peaks, peak_src):
         ring_bytes = 2 * B * Hkv * w * d * 2
         tok_s = B * world / (ms * 1e-3)
         gbs = ring_bytes / (ms * 1e-3) / 1e9
-        out[wl.name] = {"ms_per_step": ms, "tokens_per_s": tok_s, "hbm_gbs_ring": gbs,
+        out[wl.name] = {"batch": B, "ms_per_step": ms, "tokens_per_s": tok_s, "hbm_gbs_ring": gbs,
                         "hbm_frac": gbs / hbm, "hbm_peak": hbm, "peak_source": peak_src,
                         "steps": n_steps, "ring_bytes_per_step": ring_bytes}
         del cache, qs, ks, vs, pos, o
@@ -427,6 +427,11 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per GPU of the fwd+bwd layer (default: the workload's 8; "
+                         "smaller only for profiling captures)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="decode sequences (default: the workload's 64; smaller only for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
