@@ -10,19 +10,21 @@
 // visited (the band, plus the sink tile): the "Sliding Window Attention"
 // glossary's flash-attention entry (blocks outside the window are skipped).
 //
-// CTA layout (320 threads, one CTA per SM: it owns all 512 TMEM columns):
-//   warps 0-3  activation: tcgen05.ld S (one query row per thread, TMEM lane
-//              = row), add the ALiBi term, mask edge tiles, apply the
-//              activation, pack P to bf16 and tcgen05.st it over S; epilogue.
-//   warps 4-7  RoPE prep: rotate the TMA-staged Q tile and each K tile in
+// Persistent CTA (one per SM, it owns all 512 TMEM columns), warp roles:
+//   warp 0     MMA issue (one thread): S = Q'K'^T into one of NSB TMEM buffers.
+//   warp 3     MMA issue (one thread): O += P V, P read from TMEM (A operand in TMEM).
+//   warp 1     TMA producer (one thread): Q tiles, K/V tiles into a ring.
+//   warp 2     schedule (one thread): publishes each step ahead of time in a
+//              shared-memory ring read by the MMA and TMA threads.
+//   warps 4..  activation warpgroup(s) (two in sigmoid mode, taking the steps
+//              in turn): tcgen05.ld S (one query row per thread, TMEM lane =
+//              row), ALiBi term, edge-tile mask, activation, P packed to bf16
+//              and tcgen05.st over the first 64 columns of its S buffer; the
+//              epilogue of each item (O: TMEM -> bf16 global rows).
+//   last 4     RoPE prep: rotate the TMA-staged Q tile and each new K tile in
 //              place in shared memory (SWIZZLE_128B layout), then
-//              fence.proxy.async so the tensor core sees the rotated values.
-//   warp 8     MMA issue (one thread): S_b = Q K^T into TMEM buffer b = t%2,
-//              then O += P_b V with P read from TMEM (A operand in TMEM).
-//   warp 9     TMA producer (one thread): Q once, K/V tiles into a ring of
-//              NST stages.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D). P_b aliases the
-// first 64 columns of S_b (bf16 pairs).
+//              fence.proxy.async so the tensor core reads the rotated values.
+// TMEM columns: S buffers [0, 128 NSB), O0 / O1 (double-buffered per item) after them.
 #pragma once
 #include <algorithm>
 #include "common.cuh"
@@ -45,9 +47,13 @@ struct FwdTcCfg {
     static constexpr int OFF_E = OFF_V + NSLOT * TILE_BYTES;  // float2 [2][D/2]
     static constexpr int OFF_TH = OFF_E + 2 * (D / 2) * 8;    // double [D/2]
     static constexpr int OFF_BAR = OFF_TH + (D / 2) * 8;
-    static constexpr int NBAR = 6 + 4 * NSLOT + 6 + 4 + 2;
+    static constexpr int NREC = 32;                           // step records in flight (scheduler ring)
+    static constexpr int RGRP = 4;                            // records published / released per barrier
+    static constexpr int NBAR = 6 + 4 * NSLOT + 6 + 4 + 2 + 2 * (NREC / RGRP) + 3 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;         // + slack for 1024-B alignment
+    static constexpr int OFF_REC = OFF_MISC + 32;             // StepRec [NREC]
+    static constexpr int SMEM = OFF_REC + NREC * 32 + 1024;   // + slack for 1024-B alignment
+    static_assert(OFF_REC % 16 == 0 && OFF_BAR % 8 == 0, "record ring and barriers need alignment");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int NSB = (D == 64) ? 3 : 2;              // S buffers of 128 columns
     static constexpr uint32_t COL_O = NSB * 128;              // O0 at COL_O, O1 at COL_O + D
@@ -58,14 +64,17 @@ struct FwdTcCfg {
 // waits for its next tile; softmax mode keeps one, because a row's running
 // maximum and sum must live in one thread.
 // Warps 0 and 1 issue MMAs and TMA copies: the scheduler favours older
-// (lower-numbered) warps, and these two threads pace everything else.
-// Warps 2-3 are idle; activation warpgroups start at warp 4 so that warp w
-// owns TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31.
+// (lower-numbered) warps, and these threads pace everything else. Warp 2
+// walks the schedule ahead of them (StepRec ring); warp 3 issues P.V.
+// Activation warpgroups start at warp 4 so that warp w owns TMEM lanes
+// 32 (w % 4) .. 32 (w % 4) + 31.
 template <int MODE>
 struct FwdRoles {
     static constexpr int ACT_WG = (MODE == SWAT_MODE_SIGMOID_) ? 2 : 1;
     static constexpr int MMA_WARP = 0;
     static constexpr int TMA_WARP = 1;
+    static constexpr int SCHED_WARP = 2;
+    static constexpr int PV_WARP = 3;
     static constexpr int ACT_WARP0 = 4;
     static constexpr int PREP_WARP0 = ACT_WARP0 + 4 * ACT_WG;
     static constexpr int THREADS = 32 * (PREP_WARP0 + 4);
@@ -238,6 +247,47 @@ struct FwdSched {
     }
 };
 
+// One step of the schedule as the single-thread roles (MMA issue, TMA) read
+// it: a scheduler thread walks FwdSched ahead of them and publishes each step
+// in a shared-memory ring, so their own loops carry no schedule arithmetic.
+struct StepRec {
+    int step, k, b, h, kvh, i0, j0;   // step < 0: end of the schedule
+    uint32_t fl;                      // REC_* flags, slot << 8
+};
+constexpr uint32_t REC_FIRST = 1, REC_LAST = 2, REC_NEW = 4, REC_NEED_REL = 8, REC_LAST_USE = 16, REC_PAR = 32;
+
+__device__ __forceinline__ StepRec make_rec(const FwdStep &st)
+{
+    StepRec r;
+    r.step = st.step; r.k = st.k; r.b = st.b; r.h = st.h; r.kvh = st.kvh; r.i0 = st.i0; r.j0 = st.j0;
+    r.fl = (st.first ? REC_FIRST : 0u) | (st.last ? REC_LAST : 0u) | (st.is_new ? REC_NEW : 0u) |
+           (st.need_release ? REC_NEED_REL : 0u) | (st.last_use ? REC_LAST_USE : 0u) | (st.par ? REC_PAR : 0u) |
+           ((uint32_t)st.slot << 8);
+    return r;
+}
+
+__device__ __forceinline__ void rec_store(StepRec *ring, int rs, const StepRec &r)
+{
+    int4 *p = reinterpret_cast<int4 *>(ring + rs);
+    p[0] = make_int4(r.step, r.k, r.b, r.h);
+    p[1] = make_int4(r.kvh, r.i0, r.j0, (int)r.fl);
+}
+
+// Reads record idx. Records are published and released in groups of rgrp:
+// a consumer waits once per group (an mbarrier wait costs about as much as
+// an MMA, so per-record waits would starve the tensor pipe). False on abort.
+__device__ __forceinline__ bool rec_read(const StepRec *ring, uint64_t *full, uint64_t *free_, int nrec, int rgrp,
+                                         int idx, volatile int *abort_flag, StepRec &r)
+{
+    const int rs = idx % nrec, grp = rs / rgrp;
+    if (rs % rgrp == 0 && !sm100::mbar_wait(full + grp, (idx / nrec) & 1, abort_flag)) return false;
+    const int4 *p = reinterpret_cast<const int4 *>(ring + rs);
+    const int4 x = p[0], y = p[1];
+    r.step = x.x; r.k = x.y; r.b = x.z; r.h = x.w; r.kvh = y.x; r.i0 = y.y; r.j0 = y.z; r.fl = (uint32_t)y.w;
+    if (rs % rgrp == rgrp - 1) sm100::mbar_arrive(free_ + grp);
+    return true;
+}
+
 __device__ __forceinline__ bool named_bar_or(int id, int n, bool v)
 {
     uint32_t r;
@@ -347,12 +397,24 @@ __device__ __forceinline__ bool col_valid(const RowMask &m, int c)
     return ((c >= m.lo) & (c <= m.hi)) | (c < m.sh);
 }
 
-// Sigmoid weights of one S tile (TMEM, one row per thread) into bf16 P over
-// the first 64 columns of the same buffer. sigma(x) = 0.5 + 0.5 tanh(x / 2)
-// with x = s/sqrt(d) + slope (i - j); rd = i - j0.
-template <bool MASKED>
+// Validity of the 32 columns c0 .. c0+31 of one row as a bit mask (bit e =
+// column c0 + e): the window part [lo, hi] and the sink part [0, sh). A few
+// integer operations per 32 columns; every tile uses it, so full and edge
+// tiles run the same code (no per-element index arithmetic, one code copy).
+__device__ __forceinline__ uint32_t col_bits32(const RowMask &m, int c0)
+{
+    const int a = max(m.lo - c0, 0), z = min(m.hi - c0, 31);
+    const uint32_t mw = (a <= z) ? ((0xFFFFFFFFu >> (31 - z)) & (0xFFFFFFFFu << a)) : 0u;
+    const int sn = min(max(m.sh - c0, 0), 32);
+    const uint32_t ms = (sn >= 32) ? 0xFFFFFFFFu : ((1u << sn) - 1u);
+    return mw | ms;
+}
+
+// Sigmoid weights of 16 S columns into 8 packed bf16 pairs:
+// sigma(x) = 0.5 + 0.5 tanh(x / 2), x = s/sqrt(d) + slope (i - j); columns
+// whose bit in `m` is clear get P = 0.
 __device__ __forceinline__ void sigmoid_chunk(const uint32_t (&v)[16], uint32_t (&pk)[8], sm100::f2 bias,
-                                              sm100::f2 step2, sm100::f2 hs2, const RowMask &mk, int c0)
+                                              sm100::f2 step2, sm100::f2 hs2, uint32_t m)
 {
     const sm100::f2 half2 = {0.5f, 0.5f};
 #pragma unroll
@@ -362,51 +424,38 @@ __device__ __forceinline__ void sigmoid_chunk(const uint32_t (&v)[16], uint32_t 
         bias = sm100::add2(bias, step2);
         const sm100::f2 th = {sm100::tanh_approx(x.x), sm100::tanh_approx(x.y)};
         sm100::f2 p = sm100::fma2(th, half2, half2);
-        if (MASKED) {
-            p.x = col_valid(mk, c0 + 2 * e) ? p.x : 0.f;
-            p.y = col_valid(mk, c0 + 2 * e + 1) ? p.y : 0.f;
-        }
+        p.x = (m & (1u << (2 * e))) ? p.x : 0.f;
+        p.y = (m & (1u << (2 * e + 1))) ? p.y : 0.f;
         pk[e] = sm100::pack_bf16x2(p.x, p.y);
     }
 }
 
-// One 16-column chunk of P: skipped (P = 0) when no key of the chunk is
-// valid for any row of the warp, masked per element when some are not.
-template <bool MASKED>
+// One 16-column chunk of P: skipped (P = 0, no arithmetic) when no key of the
+// chunk is valid for any row of the warp (a warp-uniform test on the band
+// edges), otherwise computed with the row's column mask.
 __device__ __forceinline__ void sigmoid_chunk_any(const uint32_t (&v)[16], uint32_t s_addr, int c0,
                                                   sm100::f2 step2, sm100::f2 hs2, sm100::f2 nh2,
                                                   sm100::f2 hb2, const RowMask &mk, int rd_w0, int window,
                                                   int sink_cols)
 {
     uint32_t pk[8];
-    const sm100::f2 cpair = {(float)c0, (float)(c0 + 1)};
-    const sm100::f2 bias = sm100::fma2(cpair, nh2, hb2);   // 0.5 slope (i - j) for columns c0, c0+1
-    if (MASKED) {
-        const bool all_in = (c0 >= rd_w0 + 32 - window) && (c0 + 15 <= rd_w0);
-        const bool all_out = ((c0 > rd_w0 + 31) || (c0 + 15 < rd_w0 - window + 1)) && (c0 >= sink_cols);
-        if (all_out) {
+    const bool all_out = ((c0 > rd_w0 + 31) || (c0 + 15 < rd_w0 - window + 1)) && (c0 >= sink_cols);
+    if (all_out) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) pk[e] = 0u;
-        } else if (all_in) {
-            sigmoid_chunk<false>(v, pk, bias, step2, hs2, mk, c0);
-        } else {
-            sigmoid_chunk<true>(v, pk, bias, step2, hs2, mk, c0);
-        }
+        for (int e = 0; e < 8; ++e) pk[e] = 0u;
     } else {
-        sigmoid_chunk<false>(v, pk, bias, step2, hs2, mk, c0);
+        const sm100::f2 cpair = {(float)c0, (float)(c0 + 1)};
+        const sm100::f2 bias = sm100::fma2(cpair, nh2, hb2);   // 0.5 slope (i - j) for columns c0, c0+1
+        sigmoid_chunk(v, pk, bias, step2, hs2, col_bits32(mk, c0));
     }
     sm100::tmem_st8(s_addr + (c0 >> 1), pk);
 }
 
 // Sigmoid weights of one S tile (TMEM, one row per thread) into bf16 P over
-// the first 64 columns of the same buffer. sigma(x) = 0.5 + 0.5 tanh(x / 2)
-// with x = s/sqrt(d) + slope (i - j); rd = i - j0 for this thread's row and
-// rd_w0 for the warp's first row. On edge tiles each 16-column chunk is
-// classified for the whole warp: every key valid, none valid (P = 0 without
-// arithmetic), or mixed (per-element mask). The chunk loop is kept rolled
-// (two chunks per iteration for the double-buffered TMEM loads) so the hot
-// code stays small in the instruction cache.
-template <bool MASKED>
+// the first 64 columns of the same buffer; rd = i - j0 for this thread's row
+// and rd_w0 for the warp's first row. The chunk loop is kept rolled (two
+// chunks per iteration for the double-buffered TMEM loads) so the hot code
+// stays small in the instruction cache.
 __device__ __forceinline__ void act_sigmoid_tile(uint32_t s_addr, float hs, float hsl, int rd, int rd_w0, int j0,
                                                  int window, int n_sink)
 {
@@ -421,63 +470,62 @@ __device__ __forceinline__ void act_sigmoid_tile(uint32_t s_addr, float hs, floa
 #pragma unroll 1
     for (int c0 = 0; c0 < 128; c0 += 32) {
         sm100::tmem_ld16(s_addr + c0 + 16, v1);
-        sigmoid_chunk_any<MASKED>(v0, s_addr, c0, step2, hs2, nh2, hb2, mk, rd_w0, window, sink_cols);
+        sigmoid_chunk_any(v0, s_addr, c0, step2, hs2, nh2, hb2, mk, rd_w0, window, sink_cols);
         sm100::tmem_wait_ld_dep16(v1);
         if (c0 + 32 < 128) sm100::tmem_ld16(s_addr + c0 + 32, v0);
-        sigmoid_chunk_any<MASKED>(v1, s_addr, c0 + 16, step2, hs2, nh2, hb2, mk, rd_w0, window, sink_cols);
+        sigmoid_chunk_any(v1, s_addr, c0 + 16, step2, hs2, nh2, hb2, mk, rd_w0, window, sink_cols);
         if (c0 + 32 < 128) sm100::tmem_wait_ld_dep16(v0);
     }
 }
 
 // Softmax weights (log2 domain) of one S tile; returns the tile's row max
 // through `mx` in pass one and writes p = 2^(x - m_used) in pass two.
-template <bool MASKED>
+// Columns outside the key set count as -inf / P = 0 (column mask).
 __device__ __forceinline__ float act_softmax_max(uint32_t s_addr, float sc2, float sl2, int rd, int j0,
                                                  int window, int n_sink)
 {
     float mx = -INFINITY;
     const float b2 = sl2 * (float)rd;
     const RowMask mk = row_mask(rd, j0, window, n_sink);
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < 4; ++k) {
         uint32_t v[32];
         sm100::tmem_ld32(s_addr + 32 * k, v);
+        const uint32_t m = col_bits32(mk, 32 * k);
+        const float bk = fmaf(-sl2, (float)(32 * k), b2);
         sm100::tmem_wait_ld_dep(v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-            const int c = 32 * k + e;
-            float x = fmaf(__uint_as_float(v[e]), sc2, fmaf(-sl2, (float)c, b2));
-            if (MASKED) x = col_valid(mk, c) ? x : -INFINITY;
+            float x = fmaf(__uint_as_float(v[e]), sc2, fmaf(-sl2, (float)e, bk));
+            x = (m & (1u << e)) ? x : -INFINITY;
             mx = fmaxf(mx, x);
         }
     }
     return mx;
 }
 
-template <bool MASKED>
 __device__ __forceinline__ float act_softmax_p(uint32_t s_addr, float sc2, float sl2, int rd, int j0,
                                                int window, int n_sink, float m_used)
 {
     float lsum = 0.f;
     const float b2 = sl2 * (float)rd;
     const RowMask mk = row_mask(rd, j0, window, n_sink);
-#pragma unroll
+    const bool live = m_used != -INFINITY;
+#pragma unroll 1
     for (int k = 0; k < 4; ++k) {
         uint32_t v[32];
         sm100::tmem_ld32(s_addr + 32 * k, v);
+        const uint32_t m = live ? col_bits32(mk, 32 * k) : 0u;
+        const float bk = fmaf(-sl2, (float)(32 * k), b2);
         sm100::tmem_wait_ld_dep(v);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            const int c0 = 32 * k + 2 * e;
-            float x0 = fmaf(__uint_as_float(v[2 * e]), sc2, fmaf(-sl2, (float)c0, b2));
-            float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sc2, fmaf(-sl2, (float)(c0 + 1), b2));
-            float p0 = (m_used == -INFINITY) ? 0.f : sm100::ex2_approx(x0 - m_used);
-            float p1 = (m_used == -INFINITY) ? 0.f : sm100::ex2_approx(x1 - m_used);
-            if (MASKED) {
-                p0 = col_valid(mk, c0) ? p0 : 0.f;
-                p1 = col_valid(mk, c0 + 1) ? p1 : 0.f;
-            }
+            const float x0 = fmaf(__uint_as_float(v[2 * e]), sc2, fmaf(-sl2, (float)(2 * e), bk));
+            const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sc2, fmaf(-sl2, (float)(2 * e + 1), bk));
+            float p0 = sm100::ex2_approx(x0 - m_used), p1 = sm100::ex2_approx(x1 - m_used);
+            p0 = (m & (1u << (2 * e))) ? p0 : 0.f;
+            p1 = (m & (1u << (2 * e + 1))) ? p1 : 0.f;
             lsum += p0 + p1;
             pk[e] = sm100::pack_bf16x2(p0, p1);
         }
@@ -510,6 +558,10 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint64_t *s_full = release + NS, *p_full = s_full + NSB;
     uint64_t *o_full = p_full + NSB, *o_free = o_full + 2;
     uint64_t *o_upd = o_free + 2, *drain = o_upd + 1;
+    constexpr int NREC = C::NREC, RGRP = C::RGRP;
+    uint64_t *rec_full = drain + 1, *rec_free = rec_full + NREC / RGRP;
+    uint64_t *pv_done = rec_free + NREC / RGRP, *drain_pv = pv_done + 3;
+    StepRec *sRec = reinterpret_cast<StepRec *>(smem + C::OFF_REC);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -535,6 +587,12 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         sm100::mbar_init(o_upd, 1);
         sm100::mbar_init(drain, 1);
+        for (int s = 0; s < NREC / RGRP; ++s) {
+            sm100::mbar_init(rec_full + s, 1);
+            sm100::mbar_init(rec_free + s, 3);   // read by the S, P.V and TMA threads
+        }
+        for (int s = 0; s < NSB; ++s) sm100::mbar_init(pv_done + s, 1);
+        sm100::mbar_init(drain_pv, 1);
         *abort_flag = 0;
         sm100::fence_mbar_init();
     }
@@ -571,33 +629,61 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     S.init(a, NS, blockIdx.x, gridDim.x);
     FwdStep st;
 
-    if (warp == FWD_TMA_WARP) {
+    if (warp == RL::SCHED_WARP) {
+        // ------------------------------------------------------------ scheduler
+        if (lane == 0) {
+            for (int idx = 0;; ++idx) {
+                const bool more = S.next_step(st);
+                const int rs = idx % NREC, grp = rs / RGRP;
+                if (idx >= NREC && rs % RGRP == 0 &&
+                    !sm100::mbar_wait(rec_free + grp, ((idx / NREC) - 1) & 1, abort_flag))
+                    break;
+                StepRec r = make_rec(st);
+                if (!more) r.step = -1;
+                rec_store(sRec, rs, r);
+                if (rs % RGRP == RGRP - 1 || !more) sm100::mbar_arrive(rec_full + grp);
+                if (!more) break;
+            }
+        }
+    } else if (warp == FWD_TMA_WARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int last_par[NS];
             for (int s = 0; s < NS; ++s) last_par[s] = -1;
             int nq = 0;
-            while (S.next_step(st)) {
-                if (st.first) {
-                    const int qs = st.k & 1;
-                    if (st.k >= 2 && !sm100::mbar_wait(q_free + qs, ((st.k - 2) >> 1) & 1, abort_flag)) break;
+            StepRec r;
+            for (int idx = 0; rec_read(sRec, rec_full, rec_free, NREC, RGRP, idx, abort_flag, r) && r.step >= 0; ++idx) {
+                const int slot = (int)(r.fl >> 8), par = (r.fl & REC_PAR) ? 1 : 0;
+                if (r.fl & REC_FIRST) {
+                    const int qs = r.k & 1;
+                    if (r.k >= 2 && !sm100::mbar_wait(q_free + qs, ((r.k - 2) >> 1) & 1, abort_flag)) break;
                     sm100::mbar_arrive_expect_tx(q_full + qs, C::TILE_BYTES);
                     for (int hh = 0; hh < D / 64; ++hh)
                         sm100::tma_load_4d(sQ + qs * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_q, q_full + qs,
-                                           hh * 64, st.h, st.i0, st.b);
-                    nq = st.k + 1;
+                                           hh * 64, r.h, r.i0, r.b);
+                    // warm L2 with the next query tile of this head (a later item's Q)
+                    if (r.i0 + 128 < a.N)
+                        for (int hh = 0; hh < D / 64; ++hh) sm100::tma_prefetch_4d(&tm_q, hh * 64, r.h, r.i0 + 128, r.b);
+                    nq = r.k + 1;
                 }
-                if (st.is_new) {
-                    if (st.need_release && !sm100::mbar_wait(release + st.slot, st.par ^ 1, abort_flag)) break;
-                    sm100::mbar_arrive_expect_tx(k_full + st.slot, C::TILE_BYTES);
+                if (r.fl & REC_NEW) {
+                    if ((r.fl & REC_NEED_REL) && !sm100::mbar_wait(release + slot, par ^ 1, abort_flag)) break;
+                    sm100::mbar_arrive_expect_tx(k_full + slot, C::TILE_BYTES);
                     for (int hh = 0; hh < D / 64; ++hh)
-                        sm100::tma_load_4d(sK + st.slot * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_k,
-                                           k_full + st.slot, hh * 64, st.kvh, st.j0, st.b);
-                    sm100::mbar_arrive_expect_tx(v_full + st.slot, C::TILE_BYTES);
+                        sm100::tma_load_4d(sK + slot * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_k,
+                                           k_full + slot, hh * 64, r.kvh, r.j0, r.b);
+                    sm100::mbar_arrive_expect_tx(v_full + slot, C::TILE_BYTES);
                     for (int hh = 0; hh < D / 64; ++hh)
-                        sm100::tma_load_4d(sV + st.slot * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_v,
-                                           v_full + st.slot, hh * 64, st.kvh, st.j0, st.b);
-                    last_par[st.slot] = st.par;
+                        sm100::tma_load_4d(sV + slot * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_v,
+                                           v_full + slot, hh * 64, r.kvh, r.j0, r.b);
+                    // the next band tile usually comes next: its load then waits for a
+                    // ring slot to be released, so start it towards L2 now
+                    if (r.j0 + 128 < a.N)
+                        for (int hh = 0; hh < D / 64; ++hh) {
+                            sm100::tma_prefetch_4d(&tm_k, hh * 64, r.kvh, r.j0 + 128, r.b);
+                            sm100::tma_prefetch_4d(&tm_v, hh * 64, r.kvh, r.j0 + 128, r.b);
+                        }
+                    last_par[slot] = par;
                 }
             }
             // every issued copy must have landed before the CTA may exit
@@ -634,48 +720,28 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 sm100::mbar_arrive(k_ready + st.slot);
             }
         }
-    } else if (warp == FWD_MMA_WARP) {
+    } else if (warp == FWD_MMA_WARP || warp == RL::PV_WARP) {
         // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
+        // Two issuing threads feed the tensor pipe: warp 0 issues S = Q'K'^T,
+        // warp 3 issues O += P V. While one waits on an mbarrier the other's
+        // MMAs keep the pipe busy. S of step s reuses the TMEM buffer of step
+        // s - NSB, so it waits until that step's P.V has completed (pv_done).
+        constexpr uint32_t TILE16 = C::TILE_BYTES >> 4, HALF16 = C::HALF_BYTES >> 4;
+        auto mk = [](uint32_t hi, uint32_t lo) { return ((uint64_t)hi << 32) | lo; };
+        if (warp == FWD_MMA_WARP && lane == 0) {
             constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t IDESC_PV = sm100::idesc_bf16_f32(128, D, 0, 1);
-            // descriptor words: high half fixed per operand kind, low half = start address >> 4 (+ LBO)
             const uint64_t dq0 = sm100::sdesc_sw128(sm100::smem_u32(sQ), 16, 1024);
             const uint64_t dk0 = sm100::sdesc_sw128(sm100::smem_u32(sK), 16, 1024);
-            const uint64_t dv0 = sm100::sdesc_sw128(sm100::smem_u32(sV), C::HALF_BYTES, 1024);
-            const uint32_t hi_k = (uint32_t)(dk0 >> 32), hi_v = (uint32_t)(dv0 >> 32);
-            const uint32_t lo_q = (uint32_t)dq0, lo_k = (uint32_t)dk0, lo_v = (uint32_t)dv0;
-            constexpr uint32_t TILE16 = C::TILE_BYTES >> 4, HALF16 = C::HALF_BYTES >> 4;
-            auto mk = [](uint32_t hi, uint32_t lo) { return ((uint64_t)hi << 32) | lo; };
-            auto issue_pv = [&](const FwdStep &p) -> bool {
-                const int sb = p.step % NSB, ob = p.k & 1;
-                if (!sm100::mbar_wait(p_full + sb, (p.step / NSB) & 1, abort_flag)) return false;
-                if (p.is_new && !sm100::mbar_wait(v_full + p.slot, p.par, abort_flag)) return false;
-                if (p.first && p.k >= 2 && !sm100::mbar_wait(o_free + ob, ((p.k - 2) >> 1) & 1, abort_flag))
-                    return false;
+            const uint32_t hi_k = (uint32_t)(dk0 >> 32), lo_q = (uint32_t)dq0, lo_k = (uint32_t)dk0;
+            StepRec r;
+            for (int idx = 0;; ++idx) {
+                if (!rec_read(sRec, rec_full, rec_free, NREC, RGRP, idx, abort_flag, r) || r.step < 0) break;
+                const int qs = r.k & 1, sb = r.step % NSB, slot = (int)(r.fl >> 8);
+                if ((r.fl & REC_FIRST) && !sm100::mbar_wait(q_ready + qs, (r.k >> 1) & 1, abort_flag)) break;
+                if ((r.fl & REC_NEW) && !sm100::mbar_wait(k_ready + slot, (r.fl & REC_PAR) ? 1 : 0, abort_flag)) break;
+                if (r.step >= NSB && !sm100::mbar_wait(pv_done + sb, ((r.step / NSB) - 1) & 1, abort_flag)) break;
                 sm100::tc_fence_after();
-                const uint32_t lv = lo_v + (uint32_t)p.slot * TILE16;
-                const uint32_t d_o = tmem + C::COL_O + ob * D, a_p = tmem + sb * 128;
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    sm100::umma_ts(d_o, a_p + ks * 8, mk(hi_v, lv + ks * (2048 >> 4)), IDESC_PV,
-                                   (!p.first || ks > 0) ? 1u : 0u);
-                if (p.last_use) sm100::umma_commit(release + p.slot);
-                if (MODE == SWAT_MODE_SOFTMAX_) sm100::umma_commit(o_upd);
-                if (p.last) sm100::umma_commit(o_full + ob);
-                return true;
-            };
-            // S runs up to NSB-1 steps ahead of P.V: the S buffer of step s is
-            // reused by step s + NSB, whose S is issued after PV(s).
-            FwdStep pend0, pend1;
-            int npend = 0;
-            bool ok = true;
-            while (ok && S.next_step(st)) {
-                const int qs = st.k & 1, sb = st.step % NSB;
-                if (st.first && !sm100::mbar_wait(q_ready + qs, (st.k >> 1) & 1, abort_flag)) { ok = false; break; }
-                if (st.is_new && !sm100::mbar_wait(k_ready + st.slot, st.par, abort_flag)) { ok = false; break; }
-                sm100::tc_fence_after();
-                const uint32_t lq = lo_q + (uint32_t)qs * TILE16, lk = lo_k + (uint32_t)st.slot * TILE16;
+                const uint32_t lq = lo_q + (uint32_t)qs * TILE16, lk = lo_k + (uint32_t)slot * TILE16;
                 const uint32_t d_s = tmem + sb * 128;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
@@ -683,29 +749,82 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     sm100::umma_ss(d_s, mk(hi_k, lq + off), mk(hi_k, lk + off), IDESC_S, ks > 0 ? 1u : 0u);
                 }
                 sm100::umma_commit(s_full + sb);
-                if (st.last) sm100::umma_commit(q_free + qs);
-                if (npend == NSB - 1) {
-                    if (!issue_pv(pend0)) { ok = false; break; }
-                    pend0 = pend1;
-                    --npend;
-                }
-                if (npend == 0) pend0 = st; else pend1 = st;
-                ++npend;
+                if (r.fl & REC_LAST) sm100::umma_commit(q_free + qs);
             }
-            if (ok && npend > 0) ok = issue_pv(pend0);
-            if (ok && npend > 1) ok = issue_pv(pend1);
             sm100::umma_commit(drain);
             mbar_wait_drain(drain, 0);   // nothing of ours is in flight past this point
+        } else if (warp == RL::PV_WARP && lane == 0) {
+            constexpr uint32_t IDESC_PV = sm100::idesc_bf16_f32(128, D, 0, 1);
+            const uint64_t dv0 = sm100::sdesc_sw128(sm100::smem_u32(sV), C::HALF_BYTES, 1024);
+            const uint32_t hi_v = (uint32_t)(dv0 >> 32), lo_v = (uint32_t)dv0;
+            StepRec p;
+            for (int idx = 0;; ++idx) {
+                if (!rec_read(sRec, rec_full, rec_free, NREC, RGRP, idx, abort_flag, p) || p.step < 0) break;
+                const int sb = p.step % NSB, ob = p.k & 1, slot = (int)(p.fl >> 8);
+                const bool first = (p.fl & REC_FIRST) != 0;
+                if (!sm100::mbar_wait(p_full + sb, (p.step / NSB) & 1, abort_flag)) break;
+                if ((p.fl & REC_NEW) && !sm100::mbar_wait(v_full + slot, (p.fl & REC_PAR) ? 1 : 0, abort_flag)) break;
+                if (first && p.k >= 2 && !sm100::mbar_wait(o_free + ob, ((p.k - 2) >> 1) & 1, abort_flag)) break;
+                sm100::tc_fence_after();
+                const uint32_t lv = lo_v + (uint32_t)slot * TILE16;
+                const uint32_t d_o = tmem + C::COL_O + ob * D, a_p = tmem + sb * 128;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    sm100::umma_ts(d_o, a_p + ks * 8, mk(hi_v, lv + ks * (2048 >> 4)), IDESC_PV,
+                                   (!first || ks > 0) ? 1u : 0u);
+                sm100::umma_commit(pv_done + sb);
+                // the K tile of this step was read by S(step), complete before P(step) existed
+                if (p.fl & REC_LAST_USE) sm100::umma_commit(release + slot);
+                if (MODE == SWAT_MODE_SOFTMAX_) sm100::umma_commit(o_upd);
+                if (p.fl & REC_LAST) sm100::umma_commit(o_full + ob);
+            }
+            sm100::umma_commit(drain_pv);
+            mbar_wait_drain(drain_pv, 0);
         }
         __syncwarp();
     } else if (warp >= FWD_ACT_WARP0) {
         // ------------------------------------------------------------ activation + epilogue
+        // The epilogue of an item (O: TMEM -> bf16 global rows) is deferred to
+        // after this warpgroup's next tile: by then the item's last P.V has
+        // long completed, so the wait for O costs nothing.
         const int aw = (warp - FWD_ACT_WARP0) / 4;       // activation warpgroup
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
         const int r = 32 * (warp % 4) + lane;            // query row inside the tile (= TMEM lane)
         float m_used = -INFINITY, l_sum = 0.f;           // softmax state (log2 domain)
         const float LOG2E = 1.4426950408889634f;
-        while (S.next_step(st)) {
+        struct PendO { int k, b, h, i0; };
+        PendO pend{};
+        bool has_pend = false;
+        float pend_inv = 1.f;
+        auto epilogue = [&](const PendO &p, float inv) -> bool {
+            const int ob = p.k & 1;
+            const bool ok = sm100::mbar_wait(o_full + ob, (p.k >> 1) & 1, abort_flag);
+            if (__any_sync(0xffffffffu, !ok)) return false;
+            sm100::tc_fence_after();
+            const int i = p.i0 + r;
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)p.b * a.N + i) * a.H + p.h) * D;
+            const uint32_t o_addr = tmem + lane_base + C::COL_O + ob * D;
+#pragma unroll
+            for (int kk = 0; kk < D / 32; ++kk) {
+                uint32_t v[32];
+                sm100::tmem_ld32(o_addr + 32 * kk, v);
+                sm100::tmem_wait_ld_dep(v);
+                if (i < a.N) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = sm100::pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * kk);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+            sm100::tc_fence_before();
+            sm100::mbar_arrive(o_free + ob);
+            return true;
+        };
+        bool good = true;
+        while (good && S.next_step(st)) {
             const int sb = st.step % NSB;
             if (RL::ACT_WG == 2 && (st.step & 1) != aw) continue;   // the other warpgroup's tile
             const int i = st.i0 + r;
@@ -714,19 +833,16 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             bool ok = sm100::mbar_wait(s_full + sb, (st.step / NSB) & 1, abort_flag);
             if (__any_sync(0xffffffffu, !ok)) break;
             sm100::tc_fence_after();
-            const int j0 = st.j0, i0 = st.i0;
-            const bool masked = !(j0 + 127 <= i0 && (i0 + 127 - j0 < a.window || j0 + 127 < a.n_sink));
+            const int j0 = st.j0;
             const int rd = i - j0;
             const uint32_t s_addr = tmem + lane_base + sb * 128;
             if (MODE == SWAT_MODE_SIGMOID_) {
                 const float hs = 0.5f * a.scale, hsl = 0.5f * slope;
                 const int rd_w0 = st.i0 + 32 * (warp % 4) - j0;   // first row of this warp
-                if (masked) act_sigmoid_tile<true>(s_addr, hs, hsl, rd, rd_w0, j0, a.window, a.n_sink);
-                else act_sigmoid_tile<false>(s_addr, hs, hsl, rd, rd_w0, j0, a.window, a.n_sink);
+                act_sigmoid_tile(s_addr, hs, hsl, rd, rd_w0, j0, a.window, a.n_sink);
             } else {
                 const float sc2 = a.scale * LOG2E, sl2 = slope * LOG2E;
-                const float mx = masked ? act_softmax_max<true>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink)
-                                        : act_softmax_max<false>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink);
+                const float mx = act_softmax_max(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink);
                 // keep a stale maximum while the new one exceeds it by at most 8
                 // (weights stay <= 2^8); otherwise rescale this row of O and l
                 const bool need = mx > m_used + 8.0f;
@@ -749,45 +865,24 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (need_o) l_sum *= f;
                 }
                 if (need) m_used = mx;
-                l_sum += masked ? act_softmax_p<true>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink, m_used)
-                                : act_softmax_p<false>(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink, m_used);
+                l_sum += act_softmax_p(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink, m_used);
             }
             sm100::tmem_wait_st();
             sm100::tc_fence_before();
             sm100::mbar_arrive(p_full + sb);
+            if (has_pend) {
+                has_pend = false;
+                if (!epilogue(pend, pend_inv)) { good = false; break; }
+            }
             if (st.last) {
-                // ---- epilogue of the item: O (TMEM) -> registers -> global, one row per thread
-                const int ob = st.k & 1;
-                ok = sm100::mbar_wait(o_full + ob, (st.k >> 1) & 1, abort_flag);
-                if (__any_sync(0xffffffffu, !ok)) break;
-                sm100::tc_fence_after();
-                const float inv = (MODE == SWAT_MODE_SOFTMAX_) ? 1.f / l_sum : 1.f;
-                __nv_bfloat16 *orow =
-                    reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)st.b * a.N + i) * a.H + st.h) * D;
-                const uint32_t o_addr = tmem + lane_base + C::COL_O + ob * D;
-#pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk) {
-                    uint32_t v[32];
-                    sm100::tmem_ld32(o_addr + 32 * kk, v);
-                    sm100::tmem_wait_ld_dep(v);
-                    if (i < a.N) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            pk[e] = sm100::pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
-                                                       __uint_as_float(v[2 * e + 1]) * inv);
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * kk);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                    }
-                }
+                pend = PendO{st.k, st.b, st.h, st.i0};
+                has_pend = true;
+                pend_inv = (MODE == SWAT_MODE_SOFTMAX_) ? 1.f / l_sum : 1.f;
                 if (MODE == SWAT_MODE_SOFTMAX_ && i < a.N)
                     a.lse[((size_t)st.b * a.H + st.h) * a.N + i] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
-                sm100::tc_fence_before();
-                sm100::mbar_arrive(o_free + ob);
             }
         }
+        if (good && has_pend) epilogue(pend, pend_inv);
     }
 
     sm100::tc_fence_before();
