@@ -7,45 +7,69 @@
 //   sigmoid: dS_ij = dP_ij p_ij (1 - p_ij);  softmax: dS_ij = p_ij (dP_ij - D_i)
 //   dq'_i = sum_j dS_ij k'_j / sqrt(d),  dk'_j = sum_i dS_ij q'_i / sqrt(d),
 //   dq = R_i^T dq', dk = R_j^T dk'.
-// Two kernels, no atomics (every output row has one owner, results are
-// deterministic):
-//   dq kernel   (query tile per CTA):  S = Q'K'^T, dP = dO V^T, dS in registers,
-//                                     dQ' += dS K'          (dS as TMEM A operand)
-//   dkdv kernel (key tile per CTA, all query heads of the KV group):
-//                S^T = K'Q'^T, dP^T = V dO^T, P^T and dS^T in registers,
-//                dV += P^T dO, dK' += dS^T Q'            (TMEM A operands)
-// Roles (384 threads): warp 0 issues MMAs, warp 1 TMA copies, warps 4-7 the
-// element-wise math and the epilogue (one tile row per thread = TMEM lane),
-// warps 8-11 rotate the streamed Q or K tiles (RoPE) in shared memory.
-// TMEM: [0,128) S (its first 64 columns then hold the bf16 dS or P),
-// [128,256) dP (then dS^T in the dkdv kernel), accumulators from 256.
+// One persistent kernel template, three roles (no atomics: every output row
+// has one owner, results are deterministic):
+//   DQ    item = (b, h, 128-query tile); stationary Q', dO; streamed K', V tiles:
+//         S = Q'K'^T, dP = dO V^T, dS element-wise, dQ' += dS K'.
+//   DKDV  item = (b, kv head, 128-key tile); stationary K', V; streamed Q', dO
+//         tiles of every query head of the group: S^T = K'Q'^T, dP^T = V dO^T,
+//         dV += P^T dO, dK' += dS^T Q'.
+//   DSUM  (softmax) the DQ products without dQ': D_i = sum_j p_ij dP_ij.
+// Each streamed tile is processed as two 64-column half-steps; half h of
+// every step goes to activation warpgroup h, which owns TMEM buffer h, so the
+// element-wise work of one half overlaps the MMAs of the other.
+// Warp roles (512 threads, one CTA per SM):
+//   warp 0     issues S / dP of each half-step (X MMAs) into TMEM buffer h.
+//   warp 1     TMA: stationary tile pair per item, streamed pairs into a ring.
+//   warp 3     issues the gradient MMAs (dV, dK', dQ') of each half-step.
+//   warps 4-11 two activation warpgroups (one TMEM lane = one row per thread);
+//              the epilogue of item k runs in warpgroup k % 2, deferred until
+//              after its next half-step.
+//   warps 12-15 RoPE prep: rotate the stationary Q or K tile and each streamed
+//              K or Q tile in place in shared memory.
+// TMEM columns: [128 h, 128 h + 64) S half, [128 h + 64, 128 h + 128) dP half
+// (their first 32 columns then hold bf16 P and dS), accumulators from 256.
 #pragma once
 #include "fwd_tc.cuh"
 
 namespace swat {
 
-constexpr int BWD_MMA_WARP = 0, BWD_TMA_WARP = 1, BWD_ACT_WARP0 = 4, BWD_PREP_WARP0 = 8;
-constexpr int BWD_THREADS = 384;
+enum { BWD_ROLE_DQ = 0, BWD_ROLE_DKDV = 1, BWD_ROLE_DSUM = 2 };
 
-template <int D>
-struct BwdTcCfg {
-    static constexpr int TILE_BYTES = 128 * D * 2;
-    static constexpr int HALF_BYTES = 128 * 128;
-    static constexpr int NST = (D == 64) ? 3 : 2;          // streamed-tile stages
-    // fixed tiles (A, B) + streamed pairs (C[NST], E[NST])
-    static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + TILE_BYTES;
-    static constexpr int OFF_C = OFF_B + TILE_BYTES;
-    static constexpr int OFF_E = OFF_C + NST * TILE_BYTES;
-    static constexpr int OFF_ROT = OFF_E + NST * TILE_BYTES;  // float2 [2][D/2] bases
-    static constexpr int OFF_TH = OFF_ROT + 2 * (D / 2) * 8;  // double [D/2]
-    static constexpr int OFF_A0 = OFF_TH + (D / 2) * 8;       // float [D/2] epilogue base angle
-    static constexpr int OFF_THF = OFF_A0 + (D / 2) * 4;      // float [D/2]
-    static constexpr int OFF_ROWS = OFF_THF + (D / 2) * 4;    // float [NST][2][128] (lse, D per query)
-    static constexpr int OFF_BAR = OFF_ROWS + NST * 2 * 128 * 4;
-    static constexpr int NBAR = 2 + 4 * NST + 4;
+constexpr int BWD_X_WARP = 0, BWD_TMA_WARP = 1, BWD_G_WARP = 3, BWD_ACT_WARP0 = 4, BWD_PREP_WARP0 = 12;
+constexpr int BWD_THREADS = 512;
+
+template <int D, int ROLE>
+struct BwdCfg {
+    static constexpr int TILE = 128 * D * 2;                   // one 128-row bf16 tile
+    static constexpr int HALF_BYTES = 128 * 128;               // one 64-column SW128 box
+    static constexpr int NSTAT = (D == 64) ? 2 : 1;            // stationary tile pairs
+    static constexpr int NST = (D == 64) ? 3 : 2;              // streamed tile pairs
+    static constexpr int ACC_COLS = (ROLE == BWD_ROLE_DKDV) ? 2 * D : (ROLE == BWD_ROLE_DQ ? D : 0);
+    // bf16 P / dS of each buffer: in columns of their own when they fit next
+    // to two accumulator sets (the next S / dP MMA into the buffer then waits
+    // only for the element-wise pass, not for the gradient MMAs), else over
+    // the S / dP halves.
+    static constexpr int PD_COLS = (ROLE == BWD_ROLE_DKDV) ? 64 : (ROLE == BWD_ROLE_DQ ? 32 : 0);
+    static constexpr bool SEP_PD = PD_COLS > 0 && 256 + 2 * PD_COLS + 2 * ACC_COLS <= 512;   // keeps two accumulator sets
+    static constexpr int ACC_BASE = SEP_PD ? 256 + 2 * PD_COLS : 256;
+    static constexpr int NACC = (ACC_COLS == 0) ? 1 : ((ACC_BASE + 2 * ACC_COLS <= 512) ? 2 : 1);
+    static constexpr int OFF_A1 = 0;                           // stationary tiles [NSTAT]
+    static constexpr int OFF_A2 = OFF_A1 + NSTAT * TILE;
+    static constexpr int OFF_B1 = OFF_A2 + NSTAT * TILE;       // streamed tiles [NST]
+    static constexpr int OFF_B2 = OFF_B1 + NST * TILE;
+    static constexpr int OFF_ROT = OFF_B2 + NST * TILE;        // float2 [2][D/2] prep bases
+    static constexpr int OFF_TH = OFF_ROT + 2 * (D / 2) * 8;   // double [D/2]
+    static constexpr int OFF_THF = OFF_TH + (D / 2) * 8;       // float [D/2]
+    static constexpr int OFF_A0 = OFF_THF + (D / 2) * 4;       // float [2 wg][2][D/2] epilogue base angles
+    static constexpr int OFF_ROWS = OFF_A0 + 4 * (D / 2) * 4;  // float [2 wg][2 buf][128]: lse, D of 64 queries
+    static constexpr int OFF_DSUM = OFF_ROWS + 2 * 2 * 128 * 4; // float [2 item][2 wg][128]
+    static constexpr int OFF_BAR = OFF_DSUM + 2 * 2 * 128 * 4;
+    static constexpr int NBAR = 3 * 2 + 4 * 3 + 7 * 2 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack for 1024-B alignment
+    static_assert(OFF_BAR % 8 == 0, "barrier alignment");
+    static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
 // Inverse RoPE of one accumulator row held in TMEM (fp32, D columns), for a
@@ -84,8 +108,10 @@ __device__ __forceinline__ void unrotate_store_row(uint32_t taddr, int r, const 
     }
 }
 
-__device__ __forceinline__ void store_row_bf16_plain(uint32_t taddr, int D, __nv_bfloat16 *dst, bool store)
+template <int D>
+__device__ __forceinline__ void store_row_bf16_plain(uint32_t taddr, __nv_bfloat16 *dst, bool store)
 {
+#pragma unroll
     for (int k = 0; k < D / 32; ++k) {
         uint32_t v[32];
         sm100::tmem_ld32(taddr + 32 * k, v);
@@ -101,309 +127,7 @@ __device__ __forceinline__ void store_row_bf16_plain(uint32_t taddr, int D, __nv
     }
 }
 
-// dS of one 128x128 tile, one row per thread: reads S and dP (TMEM, fp32),
-// writes bf16 dS (scaled by 1/sqrt(d)) over the first 64 columns of the S
-// buffer (at `out_addr`), and, when `p_addr` != 0, bf16 P over another
-// buffer's first 64 columns (WRITE_P). `valid(c)` masks column c. Element-wise:
-//   sigmoid: x = s/sqrt(d) + bias_c, t = tanh(x/2), p = (1+t)/2,
-//            dS = dP (1 - t^2) / 4 / sqrt(d)
-//   softmax: p = exp(x - lse), dS = p (dP - Dr) / sqrt(d)
-template <int MODE, bool MASKED, bool WRITE_P, typename BiasF, typename ValidF, typename RowVal>
-__device__ __forceinline__ void bwd_ds_tile(uint32_t s_addr, uint32_t dp_addr, uint32_t out_addr, uint32_t p_addr,
-                                            float scale, BiasF bias_of, ValidF valid, RowVal rowval)
-{
-#pragma unroll 1
-    for (int k = 0; k < 8; ++k) {
-        uint32_t sv[16], dv[16];
-        sm100::tmem_ld16(s_addr + 16 * k, sv);
-        sm100::tmem_ld16(dp_addr + 16 * k, dv);
-        sm100::tmem_wait_ld_dep16(sv);
-        sm100::tmem_wait_ld_dep16(dv);
-        uint32_t dk[8], pkk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float ds[2], pp[2];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int c = 16 * k + 2 * e + h2;
-                const float s = __uint_as_float(sv[2 * e + h2]), dp = __uint_as_float(dv[2 * e + h2]);
-                float lse_or_zero, Dr;
-                rowval(c, lse_or_zero, Dr);
-                const float x = fmaf(s, scale, bias_of(c));
-                float p, g;
-                if (MODE == SWAT_MODE_SIGMOID_) {
-                    const float th = sm100::tanh_approx(0.5f * x);
-                    p = fmaf(0.5f, th, 0.5f);
-                    g = dp * fmaf(-th, th, 1.f) * (0.25f * scale);
-                } else {
-                    p = __expf(x - lse_or_zero);
-                    g = p * (dp - Dr) * scale;
-                }
-                if (MASKED && !valid(c)) { p = 0.f; g = 0.f; }
-                ds[h2] = g; pp[h2] = p;
-            }
-            dk[e] = sm100::pack_bf16x2(ds[0], ds[1]);
-            pkk[e] = sm100::pack_bf16x2(pp[0], pp[1]);
-        }
-        sm100::tmem_st8(out_addr + 8 * k, dk);
-        if (WRITE_P) sm100::tmem_st8(p_addr + 8 * k, pkk);
-    }
-}
-
-// Softmax row term D_i = sum_j p_ij dP_ij of one tile (fp32, masked), the
-// exact form of dO_i . o_i (it does not depend on the rounding of o).
-template <bool MASKED, typename BiasF, typename ValidF>
-__device__ __forceinline__ float bwd_rowsum_tile(uint32_t s_addr, uint32_t dp_addr, float scale, float lse,
-                                                 BiasF bias_of, ValidF valid)
-{
-    float acc = 0.f;
-#pragma unroll 1
-    for (int k = 0; k < 8; ++k) {
-        uint32_t sv[16], dv[16];
-        sm100::tmem_ld16(s_addr + 16 * k, sv);
-        sm100::tmem_ld16(dp_addr + 16 * k, dv);
-        sm100::tmem_wait_ld_dep16(sv);
-        sm100::tmem_wait_ld_dep16(dv);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int c = 16 * k + e;
-            float p = __expf(fmaf(__uint_as_float(sv[e]), scale, bias_of(c)) - lse);
-            if (MASKED && !valid(c)) p = 0.f;
-            acc = fmaf(p, __uint_as_float(dv[e]), acc);
-        }
-    }
-    return acc;
-}
-
-// ===========================================================================
-// dq kernel: one CTA per (b, h, 128-row query tile); key tiles streamed.
-// With DPASS (softmax mode, launched first) it only computes D_i into the
-// workspace: the same S and dP, no dQ' product.
-// smem A = Q (rotated), B = dO, C[] = K (rotated), E[] = V.
-// ===========================================================================
-template <int D, int MODE, bool DPASS>
-__global__ void __launch_bounds__(BWD_THREADS, 1)
-swat_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                      const BwdArgs a, float *dq_f32_unused)
-{
-    (void)dq_f32_unused;
-    using C = BwdTcCfg<D>;
-    constexpr int NST = C::NST;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = smem + C::OFF_A, *sDO = smem + C::OFF_B, *sK = smem + C::OFF_C, *sV = smem + C::OFF_E;
-    float2 *sRot = reinterpret_cast<float2 *>(smem + C::OFF_ROT);
-    double *sTh = reinterpret_cast<double *>(smem + C::OFF_TH);
-    float *sA0 = reinterpret_cast<float *>(smem + C::OFF_A0);
-    float *sThf = reinterpret_cast<float *>(smem + C::OFF_THF);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *q_full = bars, *q_ready = bars + 1;
-    uint64_t *k_full = bars + 2, *k_ready = k_full + NST, *v_full = k_ready + NST, *release = v_full + NST;
-    uint64_t *s_full = release + NST, *p_full = s_full + 1, *o_full = p_full + 1, *drain = o_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int G = a.H / a.Hkv, kvh = h / G;
-    const int i0 = qt * 128;
-    const TileRange tr = fwd_tile_range(i0, a.N, a.window, a.n_sink);
-    const int T = tr.n_tiles;
-
-    if (threadIdx.x == 0) {
-        sm100::mbar_init(q_full, 1);
-        sm100::mbar_init(q_ready, 128);
-        for (int s = 0; s < NST; ++s) {
-            sm100::mbar_init(k_full + s, 1);
-            sm100::mbar_init(k_ready + s, 128);
-            sm100::mbar_init(v_full + s, 1);
-            sm100::mbar_init(release + s, 1);
-        }
-        sm100::mbar_init(s_full, 1);
-        sm100::mbar_init(p_full, 128);
-        sm100::mbar_init(o_full, 1);
-        sm100::mbar_init(drain, 1);
-        *abort_flag = 0;
-        sm100::fence_mbar_init();
-    }
-    if (warp == BWD_MMA_WARP) {
-        sm100::tmem_alloc(tmem_slot, 512);
-        sm100::tmem_relinquish();
-    }
-    const bool is_prep = warp >= BWD_PREP_WARP0;
-    const int ptid = threadIdx.x - 32 * BWD_PREP_WARP0;
-    RotThread rot;
-    if (is_prep && a.use_rope) {
-        if (ptid < D / 2) {
-            const double th = exp2(-2.0 * (double)ptid / (double)D * a.log2_base);
-            sTh[ptid] = th;
-            sThf[ptid] = (float)th;
-            const double two_pi = 6.283185307179586476925286766559;
-            const double x = (double)i0 * th;
-            sA0[ptid] = (float)(x - rint(x / two_pi) * two_pi);
-        }
-        sm100::named_bar_sync(FWD_PREP_BAR, 128);
-        constexpr int CPR = D / 8, RS = 128 / CPR;
-        const int c = ptid % CPR, r0 = ptid / CPR;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const double th = sTh[4 * c + q];
-            const float2 w0 = rope_cs((double)r0 * th), stp = rope_cs((double)RS * th);
-            rot.w0c[q] = w0.x; rot.w0s[q] = w0.y; rot.stc[q] = stp.x; rot.sts[q] = stp.y;
-        }
-    }
-    sm100::tc_fence_before();
-    __syncthreads();
-    sm100::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == BWD_TMA_WARP) {
-        if (lane == 0) {
-            int last_par[NST];
-            for (int s = 0; s < NST; ++s) last_par[s] = -1;
-            sm100::mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
-            for (int hh = 0; hh < D / 64; ++hh) {
-                sm100::tma_load_4d(sQ + hh * C::HALF_BYTES, &tm_q, q_full, hh * 64, h, i0, b);
-                sm100::tma_load_4d(sDO + hh * C::HALF_BYTES, &tm_do, q_full, hh * 64, h, i0, b);
-            }
-            for (int t = 0; t < T; ++t) {
-                const int st = t % NST, n = t / NST;
-                if (n > 0 && !sm100::mbar_wait(release + st, (n - 1) & 1, abort_flag)) break;
-                const int j0 = fwd_tile_j0(tr, t);
-                sm100::mbar_arrive_expect_tx(k_full + st, C::TILE_BYTES);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    sm100::tma_load_4d(sK + st * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_k, k_full + st, hh * 64, kvh, j0, b);
-                sm100::mbar_arrive_expect_tx(v_full + st, C::TILE_BYTES);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    sm100::tma_load_4d(sV + st * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_v, v_full + st, hh * 64, kvh, j0, b);
-                last_par[st] = n & 1;
-            }
-            mbar_wait_drain(q_full, 0);
-            for (int s = 0; s < NST; ++s)
-                if (last_par[s] >= 0) { mbar_wait_drain(k_full + s, last_par[s]); mbar_wait_drain(v_full + s, last_par[s]); }
-        }
-    } else if (is_prep) {
-        int ebuf = 0;
-        auto make_bases = [&](int pos0) {
-            ebuf ^= 1;
-            if (a.use_rope && ptid < D / 2) sRot[ebuf * (D / 2) + ptid] = rope_cs((double)pos0 * sTh[ptid]);
-        };
-        make_bases(i0);
-        bool ok = sm100::mbar_wait(q_full, 0, abort_flag);
-        if (!named_bar_or(FWD_PREP_BAR, 128, !ok || *abort_flag)) {
-            if (a.use_rope) rope_rotate_tile<D>(sQ, sRot + ebuf * (D / 2), rot, ptid);
-            sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(q_ready);
-            for (int t = 0; t < T; ++t) {
-                const int st = t % NST, n = t / NST;
-                make_bases(fwd_tile_j0(tr, t));
-                ok = sm100::mbar_wait(k_full + st, n & 1, abort_flag);
-                if (named_bar_or(FWD_PREP_BAR, 128, !ok || *abort_flag)) break;
-                if (a.use_rope) rope_rotate_tile<D>(sK + st * C::TILE_BYTES, sRot + ebuf * (D / 2), rot, ptid);
-                sm100::fence_proxy_async_smem();
-                sm100::mbar_arrive(k_ready + st);
-            }
-        }
-    } else if (warp == BWD_MMA_WARP) {
-        if (lane == 0) {
-            constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t IDESC_DQ = sm100::idesc_bf16_f32(128, D, 0, 1);
-            const uint32_t qa = sm100::smem_u32(sQ), doa = sm100::smem_u32(sDO);
-            bool ok = sm100::mbar_wait(q_ready, 0, abort_flag);
-            for (int t = 0; ok && t < T; ++t) {
-                const int st = t % NST, n = t / NST;
-                if (!sm100::mbar_wait(k_ready + st, n & 1, abort_flag) || !sm100::mbar_wait(v_full + st, n & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                sm100::tc_fence_after();
-                const uint32_t ka = sm100::smem_u32(sK + st * C::TILE_BYTES), va = sm100::smem_u32(sV + st * C::TILE_BYTES);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
-                    sm100::umma_ss(tmem + 0, sm100::sdesc_sw128(qa + off, 16, 1024), sm100::sdesc_sw128(ka + off, 16, 1024),
-                                   IDESC_S, ks > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
-                    sm100::umma_ss(tmem + 128, sm100::sdesc_sw128(doa + off, 16, 1024), sm100::sdesc_sw128(va + off, 16, 1024),
-                                   IDESC_S, ks > 0 ? 1u : 0u);
-                }
-                sm100::umma_commit(s_full);
-                if (!sm100::mbar_wait(p_full, t & 1, abort_flag)) { ok = false; break; }
-                sm100::tc_fence_after();
-                if (!DPASS) {
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        sm100::umma_ts(tmem + 256, tmem + 0 + ks * 8, sm100::sdesc_sw128(ka + ks * 2048, C::HALF_BYTES, 1024),
-                                       IDESC_DQ, (t > 0 || ks > 0) ? 1u : 0u);
-                }
-                sm100::umma_commit(release + st);
-            }
-            if (ok) sm100::umma_commit(o_full);
-            sm100::umma_commit(drain);
-            mbar_wait_drain(drain, 0);
-        }
-        __syncwarp();
-    } else if (warp >= BWD_ACT_WARP0) {
-        const int r = 32 * (warp % 4) + lane;
-        const int i = i0 + r;
-        const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
-        const float slope = a.slopes ? __ldg(a.slopes + h) : 0.f;
-        float lse = 0.f, Dr = 0.f, dsum = 0.f;
-        if (MODE == SWAT_MODE_SOFTMAX_ && i < a.N) {
-            lse = a.lse[((size_t)b * a.H + h) * a.N + i];
-            if (!DPASS) Dr = a.Dws[((size_t)b * a.H + h) * a.N + i];
-        }
-        bool ok = sm100::mbar_wait(q_ready, 0, abort_flag);   // (also orders the epilogue's base angles)
-        for (int t = 0; ok && t < T; ++t) {
-            ok = sm100::mbar_wait(s_full, t & 1, abort_flag);
-            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-            sm100::tc_fence_after();
-            const int j0 = fwd_tile_j0(tr, t);
-            const bool masked = !(j0 + 127 <= i0 && (i0 + 127 - j0 < a.window || j0 + 127 < a.n_sink));
-            const int rd = i - j0;
-            const RowMask mk = row_mask(rd, j0, a.window, a.n_sink);
-            auto bias_of = [&](int c) { return slope * (float)(rd - c); };
-            auto valid = [&](int c) { return col_valid(mk, c); };
-            auto rowval = [&](int, float &l_, float &d_) { l_ = lse; d_ = Dr; };
-            const uint32_t s_addr = tmem + lane_base, dp_addr = tmem + lane_base + 128;
-            if (DPASS) {
-                dsum += masked ? bwd_rowsum_tile<true>(s_addr, dp_addr, a.scale, lse, bias_of, valid)
-                               : bwd_rowsum_tile<false>(s_addr, dp_addr, a.scale, lse, bias_of, valid);
-            } else if (masked) {
-                bwd_ds_tile<MODE, true, false>(s_addr, dp_addr, s_addr, 0u, a.scale, bias_of, valid, rowval);
-            } else {
-                bwd_ds_tile<MODE, false, false>(s_addr, dp_addr, s_addr, 0u, a.scale, bias_of, valid, rowval);
-            }
-            sm100::tmem_wait_st();
-            sm100::tc_fence_before();
-            sm100::mbar_arrive(p_full);
-        }
-        if (DPASS) {
-            if (ok && i < a.N) a.Dws[((size_t)b * a.H + h) * a.N + i] = dsum;
-        } else {
-            if (ok) ok = sm100::mbar_wait(o_full, 0, abort_flag);
-            if (!__any_sync(0xffffffffu, !ok)) {
-                sm100::tc_fence_after();
-                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.dq) + (((size_t)b * a.N + i) * a.H + h) * D;
-                unrotate_store_row<D>(tmem + lane_base + 256, r, sA0, sThf, a.use_rope, dst, i < a.N);
-            }
-        }
-    }
-    sm100::tc_fence_before();
-    __syncthreads();
-    sm100::tc_fence_after();
-    if (warp == BWD_MMA_WARP) sm100::tmem_dealloc(tmem, 512);
-}
-
-// ===========================================================================
-// dkdv kernel: one CTA per (b, kv head, 128-row key tile); for each query
-// head of the group, the query tiles whose key set meets this key tile.
-// smem A = K (rotated), B = V, C[] = Q (rotated), E[] = dO.
-// ===========================================================================
+// Last query tile whose key set meets key tile kt.
 __device__ __forceinline__ int bwd_q_last(int kt, int nQT, int window, int n_sink)
 {
     if (kt == 0 && n_sink > 0) return nQT - 1;            // sink keys are seen by every later query
@@ -411,78 +135,243 @@ __device__ __forceinline__ int bwd_q_last(int kt, int nQT, int window, int n_sin
     return (int)min((long long)nQT - 1, last);
 }
 
-template <int D, int MODE>
-__global__ void __launch_bounds__(BWD_THREADS, 1)
-swat_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                        const BwdArgs a)
+// Bits c0 .. c0+31 of the column interval [lo, hi] (bit e = column c0 + e).
+__device__ __forceinline__ uint32_t interval_bits32(int lo, int hi, int c0)
 {
-    using C = BwdTcCfg<D>;
-    constexpr int NST = C::NST;
+    const int a = max(lo - c0, 0), z = min(hi - c0, 31);
+    return (a <= z) ? ((0xFFFFFFFFu >> (31 - z)) & (0xFFFFFFFFu << a)) : 0u;
+}
+
+// One work item of a persistent backward CTA and its streamed tiles.
+//   DQ / DSUM: u = ((b Hkv + kvh) nQT + qt) G + g; stationary rows are the
+//              queries of (b, h = kvh G + g, qt); step t streams key tile t of
+//              the query tile's key range (fwd_tile_range).
+//   DKDV:      u = (b Hkv + kvh) nQT + kt; stationary rows are the keys of
+//              (b, kvh, kt); step t streams query tile q_first + t % per_head
+//              of query head kvh G + t / per_head.
+struct BwdItem {
+    int b, kvh, h, row0, T;
+    int q_first, per_head;     // DKDV
+    TileRange tr;              // DQ / DSUM
+};
+
+template <int ROLE>
+__device__ __forceinline__ BwdItem bwd_item(const BwdArgs &a, int u)
+{
+    BwdItem it;
+    const int G = a.H / a.Hkv, nQT = (a.N + 127) / 128;
+    const unsigned v = (unsigned)u;
+    if (ROLE == BWD_ROLE_DKDV) {
+        const unsigned kt = v % (unsigned)nQT, sq = v / (unsigned)nQT;
+        it.kvh = (int)(sq % (unsigned)a.Hkv);
+        it.b = (int)(sq / (unsigned)a.Hkv);
+        it.h = it.kvh * G;
+        it.row0 = (int)kt * 128;
+        it.q_first = (int)kt;
+        it.per_head = bwd_q_last((int)kt, nQT, a.window, a.n_sink) - (int)kt + 1;
+        it.T = G * it.per_head;
+        it.tr = TileRange{0, 0, 0};
+    } else {
+        const unsigned g = v % (unsigned)G, r = v / (unsigned)G;
+        const unsigned qt = r % (unsigned)nQT, sq = r / (unsigned)nQT;
+        it.kvh = (int)(sq % (unsigned)a.Hkv);
+        it.b = (int)(sq / (unsigned)a.Hkv);
+        it.h = it.kvh * G + (int)g;
+        it.row0 = (int)qt * 128;
+        it.tr = fwd_tile_range(it.row0, a.N, a.window, a.n_sink);
+        it.T = it.tr.n_tiles;
+        it.q_first = 0; it.per_head = 1;
+    }
+    return it;
+}
+
+// Streamed tile of step t: its head index in the streamed tensor (K/V: kv
+// head, Q/dO: query head) and its first row.
+template <int ROLE>
+__device__ __forceinline__ void bwd_stream(const BwdItem &it, int G, int t, int &head, int &pos0)
+{
+    if (ROLE == BWD_ROLE_DKDV) {
+        head = it.kvh * G + t / it.per_head;
+        pos0 = (it.q_first + t % it.per_head) * 128;
+    } else {
+        head = it.kvh;
+        pos0 = fwd_tile_j0(it.tr, t);
+    }
+}
+
+// Element-wise work of one 64-column half-step for one row (thread):
+// reads the S and dP halves from TMEM (x_addr, x_addr + 64), writes bf16 P
+// to p_addr (WRITE_P) and bf16 dS to ds_addr (WRITE_DS), 32 columns each, and
+// returns sum_c p dP (DSUM). The score of column c is
+//   sigmoid: x = s hs + hb0 + hstep c   (hs = scale/2, bias halved), t = tanh x,
+//            p = (1 + t)/2, dS = dP (1 - t^2) scale/4;
+//   softmax: x = s sc2 + b0 + bstep c - L_c  (log2 units), p = 2^x,
+//            dS = p (dP - D_c) scale,
+// with L_c, D_c per row (colL == nullptr: lrow, drow) or per column (colL,
+// colD in shared memory). Columns whose bit in m[] is clear get x = -inf,
+// hence P = 0 and dS = 0.
+template <int MODE, bool WRITE_P, bool WRITE_DS, bool DSUM>
+__device__ __forceinline__ float bwd_half_step(uint32_t x_addr, uint32_t p_addr, uint32_t ds_addr, float xs, float b0,
+                                               float bstep, const uint32_t (&m)[2], float q4, float lrow, float drow,
+                                               const float *colL, const float *colD)
+{
+    float dsum = 0.f;
+    uint32_t s0[16], d0[16], s1[16], d1[16];
+    auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dv)[16], int ch) {
+        const int c0 = 16 * ch;
+        const uint32_t mb = (m[ch >> 1] >> (c0 & 31)) & 0xFFFFu;
+        uint32_t pk[8], gk[8];
+        const sm100::f2 xs2 = {xs, xs};
+        const sm100::f2 bias0 = {fmaf(bstep, (float)c0, b0), fmaf(bstep, (float)(c0 + 1), b0)};
+        const sm100::f2 step2 = {2.f * bstep, 2.f * bstep};
+        sm100::f2 bias = bias0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const sm100::f2 sc = {__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])};
+            const sm100::f2 dp = {__uint_as_float(dv[2 * e]), __uint_as_float(dv[2 * e + 1])};
+            sm100::f2 x = sm100::fma2(sc, xs2, bias);
+            bias = sm100::add2(bias, step2);
+            x.x = (mb & (1u << (2 * e))) ? x.x : -INFINITY;
+            x.y = (mb & (1u << (2 * e + 1))) ? x.y : -INFINITY;
+            float p0, p1, g0 = 0.f, g1 = 0.f;
+            if (MODE == SWAT_MODE_SIGMOID_) {
+                const float t0 = sm100::tanh_approx(x.x), t1 = sm100::tanh_approx(x.y);
+                p0 = fmaf(0.5f, t0, 0.5f);
+                p1 = fmaf(0.5f, t1, 0.5f);
+                g0 = dp.x * (q4 * fmaf(-t0, t0, 1.f));
+                g1 = dp.y * (q4 * fmaf(-t1, t1, 1.f));
+            } else {
+                const int c = c0 + 2 * e;
+                const float L0 = colL ? colL[c] : lrow, L1 = colL ? colL[c + 1] : lrow;
+                p0 = sm100::ex2_approx(x.x - L0);
+                p1 = sm100::ex2_approx(x.y - L1);
+                if (DSUM) {
+                    dsum = fmaf(p0, dp.x, dsum);
+                    dsum = fmaf(p1, dp.y, dsum);
+                } else {
+                    const float D0 = colD ? colD[c] : drow, D1 = colD ? colD[c + 1] : drow;
+                    g0 = p0 * (dp.x - D0) * q4;
+                    g1 = p1 * (dp.y - D1) * q4;
+                }
+            }
+            if (WRITE_P) pk[e] = sm100::pack_bf16x2(p0, p1);
+            if (WRITE_DS) gk[e] = sm100::pack_bf16x2(g0, g1);
+        }
+        if (WRITE_P) sm100::tmem_st8(p_addr + 8 * ch, pk);
+        if (WRITE_DS) sm100::tmem_st8(ds_addr + 8 * ch, gk);
+    };
+    // chunks of 16 columns, two per iteration; the next chunk's TMEM loads are
+    // in flight while the current one is computed (kept rolled: small code)
+    sm100::tmem_ld16(x_addr, s0);
+    sm100::tmem_ld16(x_addr + 64, d0);
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ch += 2) {
+        sm100::tmem_wait_ld_dep16(s0);
+        sm100::tmem_wait_ld_dep16(d0);
+        sm100::tmem_ld16(x_addr + 16 * ch + 16, s1);
+        sm100::tmem_ld16(x_addr + 64 + 16 * ch + 16, d1);
+        chunk(s0, d0, ch);
+        sm100::tmem_wait_ld_dep16(s1);
+        sm100::tmem_wait_ld_dep16(d1);
+        if (ch + 2 < 4) {
+            sm100::tmem_ld16(x_addr + 16 * ch + 32, s0);
+            sm100::tmem_ld16(x_addr + 64 + 16 * ch + 32, d0);
+        }
+        chunk(s1, d1, ch + 1);
+    }
+    return dsum;
+}
+
+// ===========================================================================
+// The persistent backward kernel.
+// tm_a1/tm_a2: stationary tensors (DQ, DSUM: Q, dO; DKDV: K, V);
+// tm_b1/tm_b2: streamed tensors (DQ, DSUM: K, V; DKDV: Q, dO). Tiles a1 and
+// b1 are RoPE-rotated in shared memory.
+// ===========================================================================
+template <int D, int MODE, int ROLE>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_a2,
+                   const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
+                   const BwdArgs a)
+{
+    using C = BwdCfg<D, ROLE>;
+    constexpr int NST = C::NST, NSTAT = C::NSTAT, NACC = C::NACC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sK = smem + C::OFF_A, *sV = smem + C::OFF_B, *sQ = smem + C::OFF_C, *sDO = smem + C::OFF_E;
+    uint8_t *sA1 = smem + C::OFF_A1, *sA2 = smem + C::OFF_A2, *sB1 = smem + C::OFF_B1, *sB2 = smem + C::OFF_B2;
     float2 *sRot = reinterpret_cast<float2 *>(smem + C::OFF_ROT);
     double *sTh = reinterpret_cast<double *>(smem + C::OFF_TH);
-    float *sA0 = reinterpret_cast<float *>(smem + C::OFF_A0);
     float *sThf = reinterpret_cast<float *>(smem + C::OFF_THF);
+    float *sA0 = reinterpret_cast<float *>(smem + C::OFF_A0);
     float *sRows = reinterpret_cast<float *>(smem + C::OFF_ROWS);
+    float *sDsum = reinterpret_cast<float *>(smem + C::OFF_DSUM);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *k_full = bars, *k_ready = bars + 1;
-    uint64_t *q_full = bars + 2, *q_ready = q_full + NST, *do_full = q_ready + NST, *release = do_full + NST;
-    uint64_t *s_full = release + NST, *p_full = s_full + 1, *o_full = p_full + 1, *drain = o_full + 1;
+    uint64_t *stat_full = bars, *stat_ready = bars + 2, *stat_free = bars + 4;
+    uint64_t *b1_full = bars + 6, *b2_full = b1_full + 3, *st_ready = b2_full + 3, *st_free = st_ready + 3;
+    uint64_t *x_full = st_free + 3, *p_full = x_full + 2, *buf_free = p_full + 2, *acc_full = buf_free + 2;
+    uint64_t *acc_free = acc_full + 2, *dsum_full = acc_free + 2, *dsum_free = dsum_full + 2;
+    uint64_t *drain_x = dsum_free + 2, *drain_g = drain_x + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int kt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-    const int G = a.H / a.Hkv;
-    const int j0 = kt * 128;
-    const int nQT = (a.N + 127) / 128;
-    const int q_first = kt, q_last = bwd_q_last(kt, nQT, a.window, a.n_sink);
-    const int per_head = q_last - q_first + 1;
-    const int T = G * per_head;                           // steps: (g, query tile)
+    const int G = a.H / a.Hkv, nQT = (a.N + 127) / 128;
+    const long long U = (ROLE == BWD_ROLE_DKDV) ? (long long)a.B * a.Hkv * nQT : (long long)a.B * a.H * nQT;
+    const int u_begin = (int)(U * blockIdx.x / gridDim.x), u_end = (int)(U * (blockIdx.x + 1) / gridDim.x);
 
     if (threadIdx.x == 0) {
-        sm100::mbar_init(k_full, 1);
-        sm100::mbar_init(k_ready, 128);
-        for (int s = 0; s < NST; ++s) {
-            sm100::mbar_init(q_full + s, 1);
-            sm100::mbar_init(q_ready + s, 128);
-            sm100::mbar_init(do_full + s, 1);
-            sm100::mbar_init(release + s, 1);
+        for (int s = 0; s < 2; ++s) {
+            sm100::mbar_init(stat_full + s, 1);
+            sm100::mbar_init(stat_ready + s, 128);
+            sm100::mbar_init(stat_free + s, 1);
+            sm100::mbar_init(x_full + s, 1);
+            sm100::mbar_init(p_full + s, 128);
+            sm100::mbar_init(buf_free + s, 1);
+            sm100::mbar_init(acc_full + s, 1);
+            sm100::mbar_init(acc_free + s, 128);
+            sm100::mbar_init(dsum_full + s, 256);
+            sm100::mbar_init(dsum_free + s, 128);
         }
-        sm100::mbar_init(s_full, 1);
-        sm100::mbar_init(p_full, 128);
-        sm100::mbar_init(o_full, 1);
-        sm100::mbar_init(drain, 1);
+        for (int s = 0; s < 3; ++s) {
+            sm100::mbar_init(b1_full + s, 1);
+            sm100::mbar_init(b2_full + s, 1);
+            sm100::mbar_init(st_ready + s, 128);
+            sm100::mbar_init(st_free + s, 1);
+        }
+        sm100::mbar_init(drain_x, 1);
+        sm100::mbar_init(drain_g, 1);
         *abort_flag = 0;
         sm100::fence_mbar_init();
     }
-    if (warp == BWD_MMA_WARP) {
+    if (warp == BWD_X_WARP) {
         sm100::tmem_alloc(tmem_slot, 512);
         sm100::tmem_relinquish();
+    }
+    if (warp == BWD_TMA_WARP && lane == 0) {
+        sm100::prefetch_tmap(&tm_a1);
+        sm100::prefetch_tmap(&tm_a2);
+        sm100::prefetch_tmap(&tm_b1);
+        sm100::prefetch_tmap(&tm_b2);
     }
     const bool is_prep = warp >= BWD_PREP_WARP0;
     const int ptid = threadIdx.x - 32 * BWD_PREP_WARP0;
     RotThread rot;
-    if (is_prep && a.use_rope) {
+    if (is_prep) {
         if (ptid < D / 2) {
             const double th = exp2(-2.0 * (double)ptid / (double)D * a.log2_base);
             sTh[ptid] = th;
             sThf[ptid] = (float)th;
-            const double two_pi = 6.283185307179586476925286766559;
-            const double x = (double)j0 * th;
-            sA0[ptid] = (float)(x - rint(x / two_pi) * two_pi);
         }
         sm100::named_bar_sync(FWD_PREP_BAR, 128);
-        constexpr int CPR = D / 8, RS = 128 / CPR;
-        const int c = ptid % CPR, r0 = ptid / CPR;
+        if (a.use_rope) {
+            constexpr int CPR = D / 8, RS = 128 / CPR;
+            const int c = ptid % CPR, r0 = ptid / CPR;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const double th = sTh[4 * c + q];
-            const float2 w0 = rope_cs((double)r0 * th), stp = rope_cs((double)RS * th);
-            rot.w0c[q] = w0.x; rot.w0s[q] = w0.y; rot.stc[q] = stp.x; rot.sts[q] = stp.y;
+            for (int q = 0; q < 4; ++q) {
+                const double th = sTh[4 * c + q];
+                const float2 w0 = rope_cs((double)r0 * th), stp = rope_cs((double)RS * th);
+                rot.w0c[q] = w0.x; rot.w0s[q] = w0.y; rot.stc[q] = stp.x; rot.sts[q] = stp.y;
+            }
         }
     }
     sm100::tc_fence_before();
@@ -491,176 +380,374 @@ swat_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const uint32_t tmem = *tmem_slot;
 
     if (warp == BWD_TMA_WARP) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int last_par[NST];
-            for (int s = 0; s < NST; ++s) last_par[s] = -1;
-            sm100::mbar_arrive_expect_tx(k_full, 2 * C::TILE_BYTES);
-            for (int hh = 0; hh < D / 64; ++hh) {
-                sm100::tma_load_4d(sK + hh * C::HALF_BYTES, &tm_k, k_full, hh * 64, kvh, j0, b);
-                sm100::tma_load_4d(sV + hh * C::HALF_BYTES, &tm_v, k_full, hh * 64, kvh, j0, b);
+            int stat_par[2] = {-1, -1}, st_par[3] = {-1, -1, -1};
+            int ts = 0, k = 0;
+            bool ok = true;
+            for (int u = u_begin; ok && u < u_end; ++u, ++k) {
+                const BwdItem it = bwd_item<ROLE>(a, u);
+                const int sb = k % NSTAT;
+                if (k >= NSTAT && !sm100::mbar_wait(stat_free + sb, ((k / NSTAT) - 1) & 1, abort_flag)) break;
+                const int head_a = (ROLE == BWD_ROLE_DKDV) ? it.kvh : it.h;
+                sm100::mbar_arrive_expect_tx(stat_full + sb, 2 * C::TILE);
+                for (int hh = 0; hh < D / 64; ++hh) {
+                    sm100::tma_load_4d(sA1 + sb * C::TILE + hh * C::HALF_BYTES, &tm_a1, stat_full + sb, hh * 64, head_a, it.row0, it.b);
+                    sm100::tma_load_4d(sA2 + sb * C::TILE + hh * C::HALF_BYTES, &tm_a2, stat_full + sb, hh * 64, head_a, it.row0, it.b);
+                }
+                stat_par[sb] = (k / NSTAT) & 1;
+                for (int t = 0; t < it.T; ++t, ++ts) {
+                    const int s = ts % NST;
+                    if (ts >= NST && !sm100::mbar_wait(st_free + s, ((ts / NST) - 1) & 1, abort_flag)) { ok = false; break; }
+                    int head, pos0;
+                    bwd_stream<ROLE>(it, G, t, head, pos0);
+                    sm100::mbar_arrive_expect_tx(b1_full + s, C::TILE);
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        sm100::tma_load_4d(sB1 + s * C::TILE + hh * C::HALF_BYTES, &tm_b1, b1_full + s, hh * 64, head, pos0, it.b);
+                    sm100::mbar_arrive_expect_tx(b2_full + s, C::TILE);
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        sm100::tma_load_4d(sB2 + s * C::TILE + hh * C::HALF_BYTES, &tm_b2, b2_full + s, hh * 64, head, pos0, it.b);
+                    st_par[s] = (ts / NST) & 1;
+                }
             }
-            for (int t = 0; t < T; ++t) {
-                const int st = t % NST, n = t / NST;
-                if (n > 0 && !sm100::mbar_wait(release + st, (n - 1) & 1, abort_flag)) break;
-                const int g = t / per_head, qt = q_first + t % per_head, h = kvh * G + g;
-                sm100::mbar_arrive_expect_tx(q_full + st, C::TILE_BYTES);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    sm100::tma_load_4d(sQ + st * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_q, q_full + st, hh * 64, h, qt * 128, b);
-                sm100::mbar_arrive_expect_tx(do_full + st, C::TILE_BYTES);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    sm100::tma_load_4d(sDO + st * C::TILE_BYTES + hh * C::HALF_BYTES, &tm_do, do_full + st, hh * 64, h, qt * 128, b);
-                last_par[st] = n & 1;
-            }
-            mbar_wait_drain(k_full, 0);
-            for (int s = 0; s < NST; ++s)
-                if (last_par[s] >= 0) { mbar_wait_drain(q_full + s, last_par[s]); mbar_wait_drain(do_full + s, last_par[s]); }
+            // every issued copy must have landed before the CTA may exit
+            for (int s = 0; s < 2; ++s)
+                if (stat_par[s] >= 0) mbar_wait_drain(stat_full + s, stat_par[s]);
+            for (int s = 0; s < 3; ++s)
+                if (st_par[s] >= 0) { mbar_wait_drain(b1_full + s, st_par[s]); mbar_wait_drain(b2_full + s, st_par[s]); }
         }
     } else if (is_prep) {
+        // ------------------------------------------------------------ RoPE prep
         int ebuf = 0;
         auto make_bases = [&](int pos0) {
             ebuf ^= 1;
             if (a.use_rope && ptid < D / 2) sRot[ebuf * (D / 2) + ptid] = rope_cs((double)pos0 * sTh[ptid]);
         };
-        make_bases(j0);
-        bool ok = sm100::mbar_wait(k_full, 0, abort_flag);
-        if (!named_bar_or(FWD_PREP_BAR, 128, !ok || *abort_flag)) {
-            if (a.use_rope) rope_rotate_tile<D>(sK, sRot + ebuf * (D / 2), rot, ptid);
+        int ts = 0, k = 0;
+        bool ok = true;
+        for (int u = u_begin; ok && u < u_end; ++u, ++k) {
+            const BwdItem it = bwd_item<ROLE>(a, u);
+            const int sb = k % NSTAT;
+            make_bases(it.row0);
+            bool w_ok = sm100::mbar_wait(stat_full + sb, (k / NSTAT) & 1, abort_flag);
+            if (named_bar_or(FWD_PREP_BAR, 128, !w_ok || *abort_flag)) break;
+            if (a.use_rope) rope_rotate_tile<D>(sA1 + sb * C::TILE, sRot + ebuf * (D / 2), rot, ptid);
             sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(k_ready);
-            for (int t = 0; t < T; ++t) {
-                const int st = t % NST, n = t / NST;
-                const int qt = q_first + t % per_head;
-                make_bases(qt * 128);
-                ok = sm100::mbar_wait(q_full + st, n & 1, abort_flag);
-                if (named_bar_or(FWD_PREP_BAR, 128, !ok || *abort_flag)) break;
-                if (a.use_rope) rope_rotate_tile<D>(sQ + st * C::TILE_BYTES, sRot + ebuf * (D / 2), rot, ptid);
+            sm100::mbar_arrive(stat_ready + sb);
+            for (int t = 0; t < it.T; ++t, ++ts) {
+                const int s = ts % NST;
+                int head, pos0;
+                bwd_stream<ROLE>(it, G, t, head, pos0);
+                make_bases(pos0);
+                w_ok = sm100::mbar_wait(b1_full + s, (ts / NST) & 1, abort_flag);
+                if (named_bar_or(FWD_PREP_BAR, 128, !w_ok || *abort_flag)) { ok = false; break; }
+                if (a.use_rope) rope_rotate_tile<D>(sB1 + s * C::TILE, sRot + ebuf * (D / 2), rot, ptid);
                 sm100::fence_proxy_async_smem();
-                sm100::mbar_arrive(q_ready + st);
+                sm100::mbar_arrive(st_ready + s);
             }
         }
-    } else if (warp == BWD_MMA_WARP) {
+    } else if (warp == BWD_X_WARP) {
+        // ------------------------------------------------------------ X MMAs: S half and dP half
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t IDESC_ACC = sm100::idesc_bf16_f32(128, D, 0, 1);
-            const uint32_t ka = sm100::smem_u32(sK), va = sm100::smem_u32(sV);
-            bool ok = sm100::mbar_wait(k_ready, 0, abort_flag);
-            for (int t = 0; ok && t < T; ++t) {
-                const int st = t % NST, n = t / NST;
-                if (!sm100::mbar_wait(q_ready + st, n & 1, abort_flag) || !sm100::mbar_wait(do_full + st, n & 1, abort_flag)) {
-                    ok = false;
-                    break;
+            constexpr uint32_t IDESC_X = sm100::idesc_bf16_f32(128, 64, 0, 0);
+            const uint64_t d0 = sm100::sdesc_sw128(sm100::smem_u32(smem), 16, 1024);
+            const uint32_t hi = (uint32_t)(d0 >> 32), lo0 = (uint32_t)d0;   // lo0 + (byte offset >> 4)
+            auto dsc = [&](uint32_t off_bytes) { return ((uint64_t)hi << 32) | (lo0 + (off_bytes >> 4)); };
+            int ts = 0, k = 0, hs = 0;
+            bool ok = true;
+            for (int u = u_begin; ok && u < u_end; ++u, ++k) {
+                const BwdItem it = bwd_item<ROLE>(a, u);
+                const int sb = k % NSTAT;
+                if (!sm100::mbar_wait(stat_ready + sb, (k / NSTAT) & 1, abort_flag)) break;
+                const uint32_t a1 = C::OFF_A1 + sb * C::TILE, a2 = C::OFF_A2 + sb * C::TILE;
+                for (int t = 0; ok && t < it.T; ++t, ++ts) {
+                    const int s = ts % NST;
+                    if (!sm100::mbar_wait(st_ready + s, (ts / NST) & 1, abort_flag) ||
+                        !sm100::mbar_wait(b2_full + s, (ts / NST) & 1, abort_flag)) { ok = false; break; }
+                    const uint32_t b1 = C::OFF_B1 + s * C::TILE, b2 = C::OFF_B2 + s * C::TILE;
+                    for (int h = 0; h < 2; ++h, ++hs) {
+                        // buffer h is free again once its previous half-step's S / dP were
+                        // consumed: by the element-wise pass (P, dS elsewhere) or, when
+                        // P / dS overlay S / dP, by the gradient MMAs
+                        if (hs >= 2 && !sm100::mbar_wait(C::SEP_PD ? p_full + h : buf_free + h, ((hs >> 1) - 1) & 1,
+                                                         abort_flag)) { ok = false; break; }
+                        sm100::tc_fence_after();
+                        const uint32_t dx = tmem + h * 128;
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
+                            sm100::umma_ss(dx, dsc(a1 + off), dsc(b1 + h * 8192 + off), IDESC_X, ks > 0 ? 1u : 0u);
+                        }
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
+                            sm100::umma_ss(dx + 64, dsc(a2 + off), dsc(b2 + h * 8192 + off), IDESC_X, ks > 0 ? 1u : 0u);
+                        }
+                        sm100::umma_commit(x_full + h);
+                    }
                 }
-                sm100::tc_fence_after();
-                const uint32_t qa = sm100::smem_u32(sQ + st * C::TILE_BYTES), doa = sm100::smem_u32(sDO + st * C::TILE_BYTES);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
-                    sm100::umma_ss(tmem + 0, sm100::sdesc_sw128(ka + off, 16, 1024), sm100::sdesc_sw128(qa + off, 16, 1024),
-                                   IDESC_S, ks > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
-                    sm100::umma_ss(tmem + 128, sm100::sdesc_sw128(va + off, 16, 1024), sm100::sdesc_sw128(doa + off, 16, 1024),
-                                   IDESC_S, ks > 0 ? 1u : 0u);
-                }
-                sm100::umma_commit(s_full);
-                if (!sm100::mbar_wait(p_full, t & 1, abort_flag)) { ok = false; break; }
-                sm100::tc_fence_after();
-                // dV += P^T dO  (P^T over S columns 0..63),  dK' += dS^T Q'  (dS^T over dP columns 0..63)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    sm100::umma_ts(tmem + 256, tmem + 0 + ks * 8, sm100::sdesc_sw128(doa + ks * 2048, C::HALF_BYTES, 1024),
-                                   IDESC_ACC, (t > 0 || ks > 0) ? 1u : 0u);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    sm100::umma_ts(tmem + 256 + D, tmem + 128 + ks * 8, sm100::sdesc_sw128(qa + ks * 2048, C::HALF_BYTES, 1024),
-                                   IDESC_ACC, (t > 0 || ks > 0) ? 1u : 0u);
-                sm100::umma_commit(release + st);
+                if (ok) sm100::umma_commit(stat_free + sb);   // the item's stationary tiles are read
             }
-            if (ok) sm100::umma_commit(o_full);
-            sm100::umma_commit(drain);
-            mbar_wait_drain(drain, 0);
+            sm100::umma_commit(drain_x);
+            mbar_wait_drain(drain_x, 0);
+        }
+        __syncwarp();
+    } else if (warp == BWD_G_WARP) {
+        // ------------------------------------------------------------ gradient MMAs
+        if (lane == 0) {
+            constexpr uint32_t IDESC_G = sm100::idesc_bf16_f32(128, D, 0, 1);
+            const uint64_t d0 = sm100::sdesc_sw128(sm100::smem_u32(smem), C::HALF_BYTES, 1024);   // MN-major B
+            const uint32_t hi = (uint32_t)(d0 >> 32), lo0 = (uint32_t)d0;
+            auto dsc = [&](uint32_t off_bytes) { return ((uint64_t)hi << 32) | (lo0 + (off_bytes >> 4)); };
+            int ts = 0, k = 0, hs = 0;
+            bool ok = true;
+            for (int u = u_begin; ok && u < u_end; ++u, ++k) {
+                const BwdItem it = bwd_item<ROLE>(a, u);
+                const int ab = k % NACC;
+                const uint32_t acc = tmem + C::ACC_BASE + ab * C::ACC_COLS;
+                for (int t = 0; ok && t < it.T; ++t, ++ts) {
+                    const int s = ts % NST;
+                    const uint32_t b1 = C::OFF_B1 + s * C::TILE, b2 = C::OFF_B2 + s * C::TILE;
+                    for (int h = 0; h < 2; ++h, ++hs) {
+                        if (!sm100::mbar_wait(p_full + h, (hs >> 1) & 1, abort_flag)) { ok = false; break; }
+                        if (ROLE != BWD_ROLE_DSUM) {
+                            const bool first = (t == 0 && h == 0);
+                            if (first && k >= NACC && !sm100::mbar_wait(acc_free + ab, ((k / NACC) - 1) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            sm100::tc_fence_after();
+                            const uint32_t pa = C::SEP_PD ? tmem + 256 + h * C::PD_COLS : tmem + h * 128;
+                            const uint32_t da = C::SEP_PD ? pa + (ROLE == BWD_ROLE_DKDV ? 32 : 0) : tmem + h * 128 + 64;
+                            if (ROLE == BWD_ROLE_DKDV) {
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)    // dV += P^T dO
+                                    sm100::umma_ts(acc, pa + ks * 8, dsc(b2 + h * 8192 + ks * 2048), IDESC_G,
+                                                   (first && ks == 0) ? 0u : 1u);
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)    // dK' += dS^T Q'
+                                    sm100::umma_ts(acc + D, da + ks * 8, dsc(b1 + h * 8192 + ks * 2048), IDESC_G,
+                                                   (first && ks == 0) ? 0u : 1u);
+                            } else {
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)    // dQ' += dS K'
+                                    sm100::umma_ts(acc, da + ks * 8, dsc(b1 + h * 8192 + ks * 2048), IDESC_G,
+                                                   (first && ks == 0) ? 0u : 1u);
+                            }
+                        }
+                        sm100::umma_commit(buf_free + h);
+                        if (h == 1) sm100::umma_commit(st_free + s);   // the step's streamed tiles are read
+                        if (ROLE != BWD_ROLE_DSUM && h == 1 && t == it.T - 1) sm100::umma_commit(acc_full + ab);
+                    }
+                }
+            }
+            sm100::umma_commit(drain_g);
+            mbar_wait_drain(drain_g, 0);
         }
         __syncwarp();
     } else if (warp >= BWD_ACT_WARP0) {
-        const int r = 32 * (warp % 4) + lane;             // key row in the tile (= TMEM lane)
-        const int j = j0 + r;
+        // ------------------------------------------------------------ activation + epilogue
+        const int w = (warp - BWD_ACT_WARP0) / 4;                 // warpgroup = half of every step
+        const int r = 32 * (warp % 4) + lane;                     // stationary row (= TMEM lane)
+        const int wtid = threadIdx.x - 32 * (BWD_ACT_WARP0 + 4 * w);   // 0..127
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
-        const int atid = threadIdx.x - 32 * BWD_ACT_WARP0;   // 0..127
-        bool ok = sm100::mbar_wait(k_ready, 0, abort_flag);
-        for (int t = 0; ok && t < T; ++t) {
-            const int g = t / per_head, qt = q_first + t % per_head, h = kvh * G + g;
-            const int i0 = qt * 128;
-            float *rows = sRows + (t & 1) * 256;          // lse / D of the 128 queries of this step
-            if (MODE == SWAT_MODE_SOFTMAX_) {
-                const int iq = i0 + atid;
-                rows[atid] = iq < a.N ? a.lse[((size_t)b * a.H + h) * a.N + iq] : 0.f;
-                rows[128 + atid] = iq < a.N ? a.Dws[((size_t)b * a.H + h) * a.N + iq] : 0.f;
-                sm100::named_bar_sync(2, 128);
+        const float LOG2E = 1.4426950408889634f;
+        const bool sig = (MODE == SWAT_MODE_SIGMOID_);
+        const float xs = sig ? 0.5f * a.scale : a.scale * LOG2E;
+        const float bmul = sig ? 0.5f : LOG2E;                    // bias units
+        const float q4 = sig ? 0.25f * a.scale : a.scale;
+        struct PendE { int k, b, h, kvh, row0; };
+        PendE pend{};
+        bool has_pend = false;
+        auto epilogue = [&](const PendE &p) -> bool {
+            if (ROLE == BWD_ROLE_DSUM) {
+                const int ib = p.k & 1;
+                const bool ok = sm100::mbar_wait(dsum_full + ib, (p.k >> 1) & 1, abort_flag);
+                if (named_bar_or(2 + w, 128, !ok)) return false;
+                const float dsum = sDsum[(ib * 2 + 0) * 128 + r] + sDsum[(ib * 2 + 1) * 128 + r];
+                const int i = p.row0 + r;
+                if (i < a.N) a.Dws[((size_t)p.b * a.H + p.h) * a.N + i] = dsum;
+                sm100::mbar_arrive(dsum_free + ib);
+                return true;
             }
-            ok = sm100::mbar_wait(s_full, t & 1, abort_flag);
-            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+            const int ab = p.k % NACC;
+            const bool ok = sm100::mbar_wait(acc_full + ab, (p.k / NACC) & 1, abort_flag);
+            if (named_bar_or(2 + w, 128, !ok)) return false;
             sm100::tc_fence_after();
-            const float slope = a.slopes ? __ldg(a.slopes + h) : 0.f;
-            // column c is query i0 + c; valid iff 0 <= i - j < window, or j is a sink (j < n_sink, i >= j), and i < N
-            const int lo = j - i0;
-            const int hi = (j < a.n_sink) ? 127 : lo + a.window - 1;
-            const int hi_n = min(hi, a.N - 1 - i0);
-            const bool masked = __any_sync(0xffffffffu, !(lo <= 0 && hi_n >= 127));   // warp-uniform
-            auto bias_of = [&](int c) { return slope * (float)(c - lo); };
-            auto valid = [&](int c) { return (c >= lo) & (c <= hi_n); };
-            auto rowval = [&](int c, float &l_, float &d_) {
-                if (MODE == SWAT_MODE_SOFTMAX_) { l_ = rows[c]; d_ = rows[128 + c]; } else { l_ = 0.f; d_ = 0.f; }
-            };
-            const uint32_t s_addr = tmem + lane_base, dp_addr = tmem + lane_base + 128;
-            // dS^T over the dP buffer, P^T over the S buffer
-            if (masked) bwd_ds_tile<MODE, true, true>(s_addr, dp_addr, dp_addr, s_addr, a.scale, bias_of, valid, rowval);
-            else bwd_ds_tile<MODE, false, true>(s_addr, dp_addr, dp_addr, s_addr, a.scale, bias_of, valid, rowval);
-            sm100::tmem_wait_st();
+            float *A0 = sA0 + (w * 2 + ((p.k >> 1) & 1)) * (D / 2);
+            if (a.use_rope && wtid < D / 2) {
+                const double two_pi = 6.283185307179586476925286766559;
+                const double x = (double)p.row0 * sTh[wtid];
+                A0[wtid] = (float)(x - rint(x / two_pi) * two_pi);
+            }
+            sm100::named_bar_sync(2 + w, 128);
+            const uint32_t acc = tmem + lane_base + C::ACC_BASE + ab * C::ACC_COLS;
+            const int row = p.row0 + r;
+            if (ROLE == BWD_ROLE_DQ) {
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.dq) + (((size_t)p.b * a.N + row) * a.H + p.h) * D;
+                unrotate_store_row<D>(acc, r, A0, sThf, a.use_rope, dst, row < a.N);
+            } else {
+                const size_t o = (((size_t)p.b * a.N + row) * a.Hkv + p.kvh) * D;
+                store_row_bf16_plain<D>(acc, reinterpret_cast<__nv_bfloat16 *>(a.dv) + o, row < a.N);
+                unrotate_store_row<D>(acc + D, r, A0, sThf, a.use_rope, reinterpret_cast<__nv_bfloat16 *>(a.dk) + o,
+                                      row < a.N);
+            }
             sm100::tc_fence_before();
-            sm100::mbar_arrive(p_full);
+            sm100::mbar_arrive(acc_free + ab);
+            return true;
+        };
+        int ts = 0, k = 0;
+        bool good = true;
+        for (int u = u_begin; good && u < u_end; ++u, ++k) {
+            const BwdItem it = bwd_item<ROLE>(a, u);
+            const int row = it.row0 + r;
+            // per-row softmax terms (DQ, DSUM: the row is a query)
+            float lrow = 0.f, drow = 0.f;
+            if (!sig && ROLE != BWD_ROLE_DKDV && row < a.N) {
+                lrow = a.lse[((size_t)it.b * a.H + it.h) * a.N + row] * LOG2E;
+                if (ROLE == BWD_ROLE_DQ) drow = a.Dws[((size_t)it.b * a.H + it.h) * a.N + row];
+            }
+            float dsum = 0.f;
+            // ALiBi slope of each step's query head, loaded one step ahead
+            int head_n, pos_n;
+            bwd_stream<ROLE>(it, G, 0, head_n, pos_n);
+            float slope_n = a.slopes ? __ldg(a.slopes + (ROLE == BWD_ROLE_DKDV ? head_n : it.h)) : 0.f;
+            for (int t = 0; t < it.T; ++t, ++ts) {
+                int head, pos0;
+                bwd_stream<ROLE>(it, G, t, head, pos0);
+                const float slope = slope_n;
+                if (ROLE == BWD_ROLE_DKDV && t + 1 < it.T && a.slopes) {
+                    bwd_stream<ROLE>(it, G, t + 1, head_n, pos_n);
+                    slope_n = __ldg(a.slopes + head_n);
+                }
+                const int cb = pos0 + 64 * w;                         // first streamed row of this half
+                const float *colL = nullptr, *colD = nullptr;
+                if (!sig && ROLE == BWD_ROLE_DKDV) {
+                    // lse (log2 units) and D of the 64 queries of this half
+                    float *rows = sRows + (w * 2 + (ts & 1)) * 128;
+                    const int c = wtid & 63, iq = cb + c;
+                    float val = 0.f;
+                    if (iq < a.N) {
+                        const size_t o = ((size_t)it.b * a.H + head) * a.N + iq;
+                        val = (wtid < 64) ? a.lse[o] * LOG2E : a.Dws[o];
+                    }
+                    rows[wtid] = val;
+                    sm100::named_bar_sync(2 + w, 128);
+                    colL = rows;
+                    colD = rows + 64;
+                }
+
+                // column masks and ALiBi bias of this half
+                uint32_t m[2];
+                float b0, bstep;
+                if (ROLE == BWD_ROLE_DKDV) {
+                    const int lo = row - cb;                          // column of query i = j
+                    int hi = (row < a.n_sink) ? 63 : lo + a.window - 1;
+                    hi = min(hi, a.N - 1 - cb);
+                    m[0] = interval_bits32(lo, hi, 0);
+                    m[1] = interval_bits32(lo, hi, 32);
+                    b0 = -slope * (float)lo * bmul;                   // slope (i - j), i = cb + c
+                    bstep = slope * bmul;
+                } else {
+                    const int rd = row - cb;                          // i - j for column 0
+                    const RowMask mk = row_mask(rd, cb, a.window, a.n_sink);
+                    m[0] = col_bits32(mk, 0);
+                    m[1] = col_bits32(mk, 32);
+                    b0 = slope * (float)rd * bmul;
+                    bstep = -slope * bmul;
+                }
+                // decisions to stop are taken by the whole warpgroup (it also meets at
+                // named barriers), so no warp waits at one that the others left
+                const bool ok = sm100::mbar_wait(x_full + w, ts & 1, abort_flag);
+                if (named_bar_or(2 + w, 128, !ok)) { good = false; break; }
+                sm100::tc_fence_after();
+                if (C::SEP_PD && ts >= 1) {
+                    // P / dS columns of this buffer: read by the previous half-step's gradient MMAs
+                    const bool okp = sm100::mbar_wait(buf_free + w, (ts - 1) & 1, abort_flag);
+                    if (named_bar_or(2 + w, 128, !okp)) { good = false; break; }
+                    sm100::tc_fence_after();
+                }
+                const uint32_t x_addr = tmem + lane_base + w * 128;
+                const uint32_t p_addr = C::SEP_PD ? tmem + lane_base + 256 + w * C::PD_COLS : x_addr;
+                const uint32_t ds_addr = C::SEP_PD ? p_addr + (ROLE == BWD_ROLE_DKDV ? 32 : 0) : x_addr + 64;
+                if (ROLE == BWD_ROLE_DSUM)
+                    dsum += bwd_half_step<MODE, false, false, true>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, q4, lrow,
+                                                                    drow, colL, colD);
+                else if (ROLE == BWD_ROLE_DQ)
+                    bwd_half_step<MODE, false, true, false>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, q4, lrow, drow,
+                                                            colL, colD);
+                else
+                    bwd_half_step<MODE, true, true, false>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, q4, lrow, drow,
+                                                           colL, colD);
+                sm100::tmem_wait_st();
+                sm100::tc_fence_before();
+                sm100::mbar_arrive(p_full + w);
+                if (has_pend) {
+                    has_pend = false;
+                    if (!epilogue(pend)) { good = false; break; }
+                }
+                if (t == it.T - 1) {
+                    if (ROLE == BWD_ROLE_DSUM) {
+                        const int ib = k & 1;
+                        if (k >= 2) {
+                            const bool okf = sm100::mbar_wait(dsum_free + ib, ((k >> 1) - 1) & 1, abort_flag);
+                            if (named_bar_or(2 + w, 128, !okf)) { good = false; break; }
+                        }
+                        sDsum[(ib * 2 + w) * 128 + r] = dsum;
+                        sm100::mbar_arrive(dsum_full + ib);
+                    }
+                    if ((k & 1) == w) {
+                        pend = PendE{k, it.b, it.h, it.kvh, it.row0};
+                        has_pend = true;
+                    }
+                }
+            }
         }
-        if (ok) ok = sm100::mbar_wait(o_full, 0, abort_flag);
-        if (!__any_sync(0xffffffffu, !ok)) {
-            sm100::tc_fence_after();
-            const size_t row = ((size_t)b * a.N + j) * a.Hkv + kvh;
-            store_row_bf16_plain(tmem + lane_base + 256, D, reinterpret_cast<__nv_bfloat16 *>(a.dv) + row * D, j < a.N);
-            unrotate_store_row<D>(tmem + lane_base + 256 + D, r, sA0, sThf, a.use_rope,
-                                  reinterpret_cast<__nv_bfloat16 *>(a.dk) + row * D, j < a.N);
-        }
+        if (good && has_pend) epilogue(pend);
     }
+
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
-    if (warp == BWD_MMA_WARP) sm100::tmem_dealloc(tmem, 512);
+    if (warp == BWD_X_WARP) sm100::tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
-// Host launch
+// Host launch: persistent grids (one CTA per SM, at most one per item).
+// Softmax: DSUM (D_i into the workspace) first, then DQ and DKDV.
 // ---------------------------------------------------------------------------
+template <int D, int MODE, int ROLE>
+inline bool launch_bwd_role(const BwdArgs &a, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                            const CUtensorMap &tdo, cudaStream_t stream)
+{
+    using C = BwdCfg<D, ROLE>;
+    auto kern = swat_bwd_tc_kernel<D, MODE, ROLE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return false;
+    const long long nQT = (a.N + 127) / 128;
+    const long long U = (ROLE == BWD_ROLE_DKDV) ? (long long)a.B * a.Hkv * nQT : (long long)a.B * a.H * nQT;
+    if (U >= (1LL << 31)) return false;   // item indices are decoded in 32 bits
+    const int grid = (int)std::min<long long>(U, (long long)num_sms());
+    if (ROLE == BWD_ROLE_DKDV)
+        kern<<<grid, BWD_THREADS, C::SMEM, stream>>>(tk, tv, tq, tdo, a);
+    else
+        kern<<<grid, BWD_THREADS, C::SMEM, stream>>>(tq, tdo, tk, tv, a);
+    return true;
+}
+
 template <int D, int MODE>
 inline int launch_bwd_tc_t(const BwdArgs &a, cudaStream_t stream)
 {
-    using C = BwdTcCfg<D>;
     CUtensorMap tq, tk, tv, tdo;
     if (!make_tmap_bshd(&tq, a.q, a.B, a.N, a.H, D) || !make_tmap_bshd(&tk, a.k, a.B, a.N, a.Hkv, D) ||
         !make_tmap_bshd(&tv, a.v, a.B, a.N, a.Hkv, D) || !make_tmap_bshd(&tdo, a.dout, a.B, a.N, a.H, D))
         return -1;
-    auto kq = swat_bwd_dq_tc_kernel<D, MODE, false>;
-    auto kk = swat_bwd_dkdv_tc_kernel<D, MODE>;
-    if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return -1;
-    if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return -1;
-    const int nQT = (a.N + 127) / 128;
     int n = 0;
-    if (MODE == SWAT_MODE_SOFTMAX_) {   // D_i = sum_j p_ij dP_ij first (workspace), used by both kernels
-        auto kd = swat_bwd_dq_tc_kernel<D, MODE, true>;
-        if (cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return -1;
-        kd<<<dim3(nQT, a.H, a.B), BWD_THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, a, nullptr);
+    if (MODE == SWAT_MODE_SOFTMAX_) {
+        if (!launch_bwd_role<D, MODE, BWD_ROLE_DSUM>(a, tq, tk, tv, tdo, stream)) return -1;
         ++n;
     }
-    kq<<<dim3(nQT, a.H, a.B), BWD_THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, a, nullptr);
-    kk<<<dim3(nQT, a.Hkv, a.B), BWD_THREADS, C::SMEM, stream>>>(tq, tk, tv, tdo, a);
+    if (!launch_bwd_role<D, MODE, BWD_ROLE_DQ>(a, tq, tk, tv, tdo, stream)) return -1;
+    if (!launch_bwd_role<D, MODE, BWD_ROLE_DKDV>(a, tq, tk, tv, tdo, stream)) return -1;
     return n + 2;
 }
 
@@ -670,6 +757,7 @@ inline size_t tc_bwd_extra_workspace(int B, int H, int Hkv, int N, int d)
     return 0;
 }
 
+// Returns the number of kernels launched, or -1 on a launch-configuration error.
 inline int launch_bwd_tc(const BwdArgs &a, void *extra_ws, cudaStream_t stream)
 {
     (void)extra_ws;
