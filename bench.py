@@ -107,17 +107,23 @@ class ClockSampler:
 
 
 def dist_setup():
+    """One process per GPU: NCCL over the GPUs; gloo when no GPU is present
+    (the host-side logic is tested that way)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if cuda:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    elif cuda:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -129,13 +135,26 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time: every multi-GPU number is device-timed per
+    rank and reduced with MAX."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's own batch (independent units: no data-path collective)."""
+    return 100 * rank
+
+
+def job_value(flops_per_rank_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: the units all ranks processed over the slowest rank's time."""
+    return flops_per_rank_step * world * steps / (max_ms * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------------------
@@ -225,7 +244,7 @@ def run_swat(args):
     B, H, Hkv, N, d, w = args.batch or wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.window
     kw = dict(window=w, n_sink=0, mode=binding.MODE_SIGMOID, slopes=wl.slope_tensor(),
               rope_base=wl.rope_base)
-    q, k, v, do = [t.to(dev) for t in inputs.qkv(B, N, H, Hkv, d, seed=100 * rank, scale=wl.scale,
+    q, k, v, do = [t.to(dev) for t in inputs.qkv(B, N, H, Hkv, d, seed=rank_seed(rank), scale=wl.scale,
                                                   dtype=torch.bfloat16, with_dout=True)]
     slopes = kw["slopes"].to(dev)
     kw["slopes"] = slopes
@@ -275,7 +294,7 @@ def run_swat(args):
     ff = fwd_flops(B, H, d, N, w)
     bf = 2.5 * ff
     step_flops = ff + bf
-    value = step_flops * world * args.steps / (ms * 1e-3) / 1e12
+    value = job_value(step_flops, world, args.steps, ms)
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
@@ -342,7 +361,7 @@ def bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, k
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     nbytes = lambda ts: sum(t.numel() * t.element_size() for t in ts)
-    e2e = {"value": step_flops * world * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    e2e = {"value": job_value(step_flops, world, args.steps, e2e_ms), "unit": "TFLOP/s",
            "h2d_bytes_per_step": nbytes((hq, hk, hv, hdo)),
            "d2h_bytes_per_step": nbytes((ho, hdq, hdk, hdv))}
     return e2e
