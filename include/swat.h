@@ -141,7 +141,7 @@ SWAT_API size_t swa_decode_workspace_bytes(int B, int H, int Hkv, int d, int win
 /* Size of the library's own decode scratch buffer (16 MiB of device memory
  * per device, reserved when the library's device code is loaded). A decode
  * step fits iff swa_decode_workspace_bytes(B, H, Hkv, d, window) is at most
- * this: e.g. 64 sequences x 32 query heads, d 128, window 4096 need 8.1 MiB. */
+ * this: e.g. 64 sequences x 32 query heads, d 128, window 4096 need 2.1 MiB. */
 #define SWA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 /* swa_decode_step without a workspace argument: the same decode step, same

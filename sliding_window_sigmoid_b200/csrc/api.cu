@@ -236,11 +236,10 @@ int swa_decode_step(const void *q, const void *k_new, const void *v_new,
     a.part_l = (float *)((char *)workspace + po + pm);
     int threads_c = ((d + 31) / 32) * 32;
     if (dtype == SWAT_BF16) {
-        swat::swa_decode_write_kernel<__nv_bfloat16><<<B, 128, 0, S(stream)>>>(a);
         int m = swat::launch_decode_attn_fast(a, S(stream));
         if (m < 0) return SWAT_ERR_CUDA;
         swat::swa_decode_combine_kernel<__nv_bfloat16><<<(unsigned)rows, threads_c, 0, S(stream)>>>(a);
-        return after_launch(2 + m);
+        return after_launch(1 + m);
     }
     swat::swa_decode_write_kernel<float><<<B, 128, 0, S(stream)>>>(a);
     dim3 grid(a.nsplit, B * Hkv);

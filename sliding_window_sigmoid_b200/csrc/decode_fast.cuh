@@ -42,6 +42,39 @@ swa_decode_attn_bf16_kernel(DecArgs a)
     const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(a.k_cache) + ((size_t)b * a.Hkv + kvh) * (size_t)w * D;
     const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(a.v_cache) + ((size_t)b * a.Hkv + kvh) * (size_t)w * D;
 
+    // The new token first: the CTA whose slot range holds slot P mod w rotates
+    // k_new at P and stores it and v_new there (and in sink slot P when
+    // P < n_sink), the same values the separate write kernel stores, then
+    // syncs so that its own reads below see them. No other CTA reads that slot.
+    if (P < 0) {
+        if (split == 0 && threadIdx.x == 0) record_status(-1);   // positions are absolute, >= 0
+    } else if ((int)(P % w) >= s0 && (int)(P % w) < s1) {
+        const int slot = (int)(P % w);
+        const __nv_bfloat16 *kt = reinterpret_cast<const __nv_bfloat16 *>(a.k_new) + ((size_t)b * a.Hkv + kvh) * D;
+        const __nv_bfloat16 *vt = reinterpret_cast<const __nv_bfloat16 *>(a.v_new) + ((size_t)b * a.Hkv + kvh) * D;
+        __nv_bfloat16 *kw = const_cast<__nv_bfloat16 *>(kc) + (size_t)slot * D;
+        __nv_bfloat16 *vw = const_cast<__nv_bfloat16 *>(vc) + (size_t)slot * D;
+        for (int t = threadIdx.x; t < D / 2; t += blockDim.x) {
+            const float x0 = __bfloat162float(kt[2 * t]), x1 = __bfloat162float(kt[2 * t + 1]);
+            float y0 = x0, y1 = x1;
+            if (a.use_rope) {
+                float c, sn;
+                rope_cos_sin(P, rope_theta(t, D, a.log2_base), c, sn);
+                rope_pair(x0, x1, c, sn, y0, y1);
+            }
+            const __nv_bfloat16 k0 = __float2bfloat16(y0), k1 = __float2bfloat16(y1);
+            kw[2 * t] = k0; kw[2 * t + 1] = k1;
+            vw[2 * t] = vt[2 * t]; vw[2 * t + 1] = vt[2 * t + 1];
+            if (P < a.n_sink) {
+                const size_t sb = (((size_t)b * a.Hkv + kvh) * a.n_sink + (size_t)P) * D + 2 * t;
+                __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(a.k_sink), *vs = reinterpret_cast<__nv_bfloat16 *>(a.v_sink);
+                ks[sb] = k0; ks[sb + 1] = k1;
+                vs[sb] = vt[2 * t]; vs[sb + 1] = vt[2 * t + 1];
+            }
+        }
+        __syncthreads();
+    }
+
     // ---- rotated queries of the group, this lane's 8 dimensions
     float q[G][8];
     {
@@ -256,8 +289,10 @@ inline bool launch_decode_attn_dg(const DecArgs &a, cudaStream_t stream, int G)
     }
 }
 
-// bf16 decode attention: the streaming kernel for d in {64, 128} and a group
-// of 1, 2, 4 or 8 query heads per KV head; the generic kernel otherwise.
+// bf16 decode step up to the combine: the streaming kernel (which also stores
+// the new token) for d in {64, 128} and a group of 1, 2, 4 or 8 query heads
+// per KV head; the write kernel and the generic kernel otherwise. Returns the
+// number of kernels launched.
 inline int launch_decode_attn_fast(const DecArgs &a, cudaStream_t stream)
 {
     const int G = a.H / a.Hkv;
@@ -268,9 +303,11 @@ inline int launch_decode_attn_fast(const DecArgs &a, cudaStream_t stream)
     else if (a.d == 64)
         done = a.mode == SWAT_MODE_SIGMOID_ ? launch_decode_attn_dg<64, SWAT_MODE_SIGMOID_>(a, stream, G)
                                             : launch_decode_attn_dg<64, SWAT_MODE_SOFTMAX_>(a, stream, G);
-    if (!done) {
+    if (!done) {   // the generic kernel expects the new token already in the ring
+        swa_decode_write_kernel<__nv_bfloat16><<<a.B, 128, 0, stream>>>(a);
         dim3 grid(a.nsplit, a.B * a.Hkv);
         swa_decode_attn_generic_kernel<__nv_bfloat16><<<grid, DEC_THREADS, 0, stream>>>(a);
+        return 2;
     }
     return 1;
 }
