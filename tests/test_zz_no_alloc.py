@@ -19,7 +19,7 @@ FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: rejected before any laun
 
 def test_noalloc_rejects_too_large_before_any_launch():
     L = binding.lib()
-    B, H, Hkv, d, w = 512, 32, 8, 128, 4096
+    B, H, Hkv, d, w = 2048, 32, 8, 128, 4096
     assert L.swa_decode_workspace_bytes(B, H, Hkv, d, w) > binding.NOALLOC_SCRATCH_BYTES
     n0 = binding.launch_count()
     st = L.swa_decode_step_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
