@@ -77,7 +77,7 @@ struct BwdCfg {
 // position pos0 reduced in fp64), reduced again in fp32 before __sincosf.
 template <int D>
 __device__ __forceinline__ void unrotate_store_row(uint32_t taddr, int r, const float *A0, const float *THF,
-                                                   bool use_rope, __nv_bfloat16 *dst, bool store)
+                                                   bool use_rope, __nv_bfloat16 *dst, bool store, float mul = 1.f)
 {
     const float two_pi = 6.2831853071795865f, inv_two_pi = 0.15915494309189534f;
 #pragma unroll
@@ -88,7 +88,7 @@ __device__ __forceinline__ void unrotate_store_row(uint32_t taddr, int r, const 
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+            float x0 = __uint_as_float(v[2 * e]) * mul, x1 = __uint_as_float(v[2 * e + 1]) * mul;
             if (use_rope) {
                 const int t = 16 * k + e;
                 float ang = fmaf((float)r, THF[t], A0[t]);
@@ -201,83 +201,91 @@ __device__ __forceinline__ void bwd_stream(const BwdItem &it, int G, int t, int 
 
 // Element-wise work of one 64-column half-step for one row (thread):
 // reads the S and dP halves from TMEM (x_addr, x_addr + 64), writes bf16 P
-// to p_addr (WRITE_P) and bf16 dS to ds_addr (WRITE_DS), 32 columns each, and
+// to p_addr (WRITE_P) and bf16 g to ds_addr (WRITE_DS), 32 columns each, and
 // returns sum_c p dP (DSUM). The score of column c is
 //   sigmoid: x = s hs + hb0 + hstep c   (hs = scale/2, bias halved), t = tanh x,
-//            p = (1 + t)/2, dS = dP (1 - t^2) scale/4;
+//            p = (1 + t)/2, g = dP p (1 - p);
 //   softmax: x = s sc2 + b0 + bstep c - L_c  (log2 units), p = 2^x,
-//            dS = p (dP - D_c) scale,
+//            g = p (dP - D_c),
 // with L_c, D_c per row (colL == nullptr: lrow, drow) or per column (colL,
-// colD in shared memory). Columns whose bit in m[] is clear get x = -inf,
-// hence P = 0 and dS = 0.
+// colD in shared memory); dS = g scale, the factor applied to the dQ' / dK'
+// accumulators in the epilogue. Columns whose bit in m[] is clear get
+// x = -inf, hence P = 0 and g = 0. Each 32-column block computes all its
+// scores, then all its MUFU results, then the rest, so the MUFU work of one
+// column overlaps the FMA work of others.
 template <int MODE, bool WRITE_P, bool WRITE_DS, bool DSUM>
 __device__ __forceinline__ float bwd_half_step(uint32_t x_addr, uint32_t p_addr, uint32_t ds_addr, float xs, float b0,
-                                               float bstep, const uint32_t (&m)[2], float q4, float lrow, float drow,
+                                               float bstep, const uint32_t (&m)[2], float lrow, float drow,
                                                const float *colL, const float *colD)
 {
     float dsum = 0.f;
-    uint32_t s0[16], d0[16], s1[16], d1[16];
-    auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dv)[16], int ch) {
-        const int c0 = 16 * ch;
-        const uint32_t mb = (m[ch >> 1] >> (c0 & 31)) & 0xFFFFu;
-        uint32_t pk[8], gk[8];
+#pragma unroll 1
+    for (int cc = 0; cc < 2; ++cc) {
+        uint32_t s0[16], s1[16], d0[16], d1[16];
+        sm100::tmem_ld16(x_addr + 32 * cc, s0);
+        sm100::tmem_ld16(x_addr + 32 * cc + 16, s1);
+        sm100::tmem_ld16(x_addr + 64 + 32 * cc, d0);
+        sm100::tmem_ld16(x_addr + 64 + 32 * cc + 16, d1);
+        const int c0 = 32 * cc;
+        const uint32_t mb = m[cc];
         const sm100::f2 xs2 = {xs, xs};
-        const sm100::f2 bias0 = {fmaf(bstep, (float)c0, b0), fmaf(bstep, (float)(c0 + 1), b0)};
         const sm100::f2 step2 = {2.f * bstep, 2.f * bstep};
-        sm100::f2 bias = bias0;
+        sm100::f2 bias2 = {fmaf(bstep, (float)c0, b0), fmaf(bstep, (float)(c0 + 1), b0)};
+        sm100::tmem_wait_ld_dep16(s0);
+        sm100::tmem_wait_ld_dep16(s1);
+        sm100::tmem_wait_ld_dep16(d0);
+        sm100::tmem_wait_ld_dep16(d1);
+        // scores (masked columns: -inf)
+        float x[32];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const sm100::f2 sc = {__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])};
-            const sm100::f2 dp = {__uint_as_float(dv[2 * e]), __uint_as_float(dv[2 * e + 1])};
-            sm100::f2 x = sm100::fma2(sc, xs2, bias);
-            bias = sm100::add2(bias, step2);
-            x.x = (mb & (1u << (2 * e))) ? x.x : -INFINITY;
-            x.y = (mb & (1u << (2 * e + 1))) ? x.y : -INFINITY;
-            float p0, p1, g0 = 0.f, g1 = 0.f;
+        for (int e = 0; e < 16; ++e) {
+            const uint32_t *sv = e < 8 ? s0 : s1;
+            const int k = e & 7;
+            const sm100::f2 xx = sm100::fma2({__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])}, xs2, bias2);
+            bias2 = sm100::add2(bias2, step2);
+            x[2 * e] = xx.x;
+            x[2 * e + 1] = xx.y;
+        }
+        if (MODE != SWAT_MODE_SIGMOID_) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] -= colL ? colL[c0 + e] : lrow;
+        }
+        if (!__all_sync(0xffffffffu, mb == 0xFFFFFFFFu)) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = (mb & (1u << e)) ? x[e] : -INFINITY;
+        }
+        // MUFU: t = tanh x (sigmoid) or p = 2^x (softmax)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = (MODE == SWAT_MODE_SIGMOID_) ? sm100::tanh_approx(x[e]) : sm100::ex2_approx(x[e]);
+        uint32_t pk[16], gk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const uint32_t *dv = e < 8 ? d0 : d1;
+            const int k = e & 7;
+            const sm100::f2 dp = {__uint_as_float(dv[2 * k]), __uint_as_float(dv[2 * k + 1])};
+            sm100::f2 p, g;
             if (MODE == SWAT_MODE_SIGMOID_) {
-                const float t0 = sm100::tanh_approx(x.x), t1 = sm100::tanh_approx(x.y);
-                p0 = fmaf(0.5f, t0, 0.5f);
-                p1 = fmaf(0.5f, t1, 0.5f);
-                g0 = dp.x * (q4 * fmaf(-t0, t0, 1.f));
-                g1 = dp.y * (q4 * fmaf(-t1, t1, 1.f));
+                const sm100::f2 t = {x[2 * e], x[2 * e + 1]};
+                p = sm100::fma2(t, {0.5f, 0.5f}, {0.5f, 0.5f});
+                const sm100::f2 q = sm100::fma2(t, {-0.5f, -0.5f}, {0.5f, 0.5f});
+                g = sm100::mul2(dp, sm100::mul2(p, q));
             } else {
-                const int c = c0 + 2 * e;
-                const float L0 = colL ? colL[c] : lrow, L1 = colL ? colL[c + 1] : lrow;
-                p0 = sm100::ex2_approx(x.x - L0);
-                p1 = sm100::ex2_approx(x.y - L1);
+                p = {x[2 * e], x[2 * e + 1]};
                 if (DSUM) {
-                    dsum = fmaf(p0, dp.x, dsum);
-                    dsum = fmaf(p1, dp.y, dsum);
+                    dsum = fmaf(p.x, dp.x, dsum);
+                    dsum = fmaf(p.y, dp.y, dsum);
+                    g = {0.f, 0.f};
                 } else {
-                    const float D0 = colD ? colD[c] : drow, D1 = colD ? colD[c + 1] : drow;
-                    g0 = p0 * (dp.x - D0) * q4;
-                    g1 = p1 * (dp.y - D1) * q4;
+                    const int c = c0 + 2 * e;
+                    const sm100::f2 dd = {colD ? colD[c] : drow, colD ? colD[c + 1] : drow};
+                    g = sm100::mul2(p, sm100::add2(dp, {-dd.x, -dd.y}));
                 }
             }
-            if (WRITE_P) pk[e] = sm100::pack_bf16x2(p0, p1);
-            if (WRITE_DS) gk[e] = sm100::pack_bf16x2(g0, g1);
+            if (WRITE_P) pk[e] = sm100::pack_bf16x2(p.x, p.y);
+            if (WRITE_DS) gk[e] = sm100::pack_bf16x2(g.x, g.y);
         }
-        if (WRITE_P) sm100::tmem_st8(p_addr + 8 * ch, pk);
-        if (WRITE_DS) sm100::tmem_st8(ds_addr + 8 * ch, gk);
-    };
-    // chunks of 16 columns, two per iteration; the next chunk's TMEM loads are
-    // in flight while the current one is computed (kept rolled: small code)
-    sm100::tmem_ld16(x_addr, s0);
-    sm100::tmem_ld16(x_addr + 64, d0);
-#pragma unroll 1
-    for (int ch = 0; ch < 4; ch += 2) {
-        sm100::tmem_wait_ld_dep16(s0);
-        sm100::tmem_wait_ld_dep16(d0);
-        sm100::tmem_ld16(x_addr + 16 * ch + 16, s1);
-        sm100::tmem_ld16(x_addr + 64 + 16 * ch + 16, d1);
-        chunk(s0, d0, ch);
-        sm100::tmem_wait_ld_dep16(s1);
-        sm100::tmem_wait_ld_dep16(d1);
-        if (ch + 2 < 4) {
-            sm100::tmem_ld16(x_addr + 16 * ch + 32, s0);
-            sm100::tmem_ld16(x_addr + 64 + 16 * ch + 32, d0);
-        }
-        chunk(s1, d1, ch + 1);
+        if (WRITE_P) sm100::tmem_st16(p_addr + 16 * cc, pk);
+        if (WRITE_DS) sm100::tmem_st16(ds_addr + 16 * cc, gk);
     }
     return dsum;
 }
@@ -555,7 +563,6 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
         const bool sig = (MODE == SWAT_MODE_SIGMOID_);
         const float xs = sig ? 0.5f * a.scale : a.scale * LOG2E;
         const float bmul = sig ? 0.5f : LOG2E;                    // bias units
-        const float q4 = sig ? 0.25f * a.scale : a.scale;
         struct PendE { int k, b, h, kvh, row0; };
         PendE pend{};
         bool has_pend = false;
@@ -585,12 +592,12 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             const int row = p.row0 + r;
             if (ROLE == BWD_ROLE_DQ) {
                 __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.dq) + (((size_t)p.b * a.N + row) * a.H + p.h) * D;
-                unrotate_store_row<D>(acc, r, A0, sThf, a.use_rope, dst, row < a.N);
+                unrotate_store_row<D>(acc, r, A0, sThf, a.use_rope, dst, row < a.N, a.scale);   // dS = g scale
             } else {
                 const size_t o = (((size_t)p.b * a.N + row) * a.Hkv + p.kvh) * D;
                 store_row_bf16_plain<D>(acc, reinterpret_cast<__nv_bfloat16 *>(a.dv) + o, row < a.N);
                 unrotate_store_row<D>(acc + D, r, A0, sThf, a.use_rope, reinterpret_cast<__nv_bfloat16 *>(a.dk) + o,
-                                      row < a.N);
+                                      row < a.N, a.scale);
             }
             sm100::tc_fence_before();
             sm100::mbar_arrive(acc_free + ab);
@@ -671,13 +678,13 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                 const uint32_t p_addr = C::SEP_PD ? tmem + lane_base + 256 + w * C::PD_COLS : x_addr;
                 const uint32_t ds_addr = C::SEP_PD ? p_addr + (ROLE == BWD_ROLE_DKDV ? 32 : 0) : x_addr + 64;
                 if (ROLE == BWD_ROLE_DSUM)
-                    dsum += bwd_half_step<MODE, false, false, true>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, q4, lrow,
+                    dsum += bwd_half_step<MODE, false, false, true>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, lrow,
                                                                     drow, colL, colD);
                 else if (ROLE == BWD_ROLE_DQ)
-                    bwd_half_step<MODE, false, true, false>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, q4, lrow, drow,
+                    bwd_half_step<MODE, false, true, false>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, lrow, drow,
                                                             colL, colD);
                 else
-                    bwd_half_step<MODE, true, true, false>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, q4, lrow, drow,
+                    bwd_half_step<MODE, true, true, false>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, lrow, drow,
                                                            colL, colD);
                 sm100::tmem_wait_st();
                 sm100::tc_fence_before();
