@@ -44,15 +44,20 @@ struct BwdCfg {
     static constexpr int TILE = 128 * D * 2;                   // one 128-row bf16 tile
     static constexpr int HALF_BYTES = 128 * 128;               // one 64-column SW128 box
     static constexpr int NSTAT = (D == 64) ? 2 : 1;            // stationary tile pairs
-    static constexpr int NST = (D == 64) ? 3 : 2;              // streamed tile pairs
+    static constexpr int NST = (D == 64) ? 4 : 2;              // streamed tile pairs
     static constexpr int ACC_COLS = (ROLE == BWD_ROLE_DKDV) ? 2 * D : (ROLE == BWD_ROLE_DQ ? D : 0);
     // bf16 P / dS of each buffer: in columns of their own when they fit next
     // to two accumulator sets (the next S / dP MMA into the buffer then waits
     // only for the element-wise pass, not for the gradient MMAs), else over
     // the S / dP halves.
+    // TMEM buffers of S / dP halves (128 columns each) in flight: three where
+    // they fit next to two accumulator sets (the dependency chain of a buffer
+    // -- S / dP MMAs, element-wise pass, gradient MMAs -- then spans three
+    // half-steps), else two.
+    static constexpr int NBUF = (3 * 128 + 2 * ACC_COLS <= 512 && ROLE != BWD_ROLE_DSUM) ? 3 : 2;
     static constexpr int PD_COLS = (ROLE == BWD_ROLE_DKDV) ? 64 : (ROLE == BWD_ROLE_DQ ? 32 : 0);
-    static constexpr bool SEP_PD = PD_COLS > 0 && 256 + 2 * PD_COLS + 2 * ACC_COLS <= 512;   // keeps two accumulator sets
-    static constexpr int ACC_BASE = SEP_PD ? 256 + 2 * PD_COLS : 256;
+    static constexpr bool SEP_PD = NBUF == 2 && PD_COLS > 0 && 256 + 2 * PD_COLS + 2 * ACC_COLS <= 512;
+    static constexpr int ACC_BASE = NBUF * 128 + (SEP_PD ? 2 * PD_COLS : 0);
     static constexpr int NACC = (ACC_COLS == 0) ? 1 : ((ACC_BASE + 2 * ACC_COLS <= 512) ? 2 : 1);
     static constexpr int OFF_A1 = 0;                           // stationary tiles [NSTAT]
     static constexpr int OFF_A2 = OFF_A1 + NSTAT * TILE;
@@ -65,11 +70,12 @@ struct BwdCfg {
     static constexpr int OFF_ROWS = OFF_A0 + 4 * (D / 2) * 4;  // float [2 wg][2 buf][128]: lse, D of 64 queries
     static constexpr int OFF_DSUM = OFF_ROWS + 2 * 2 * 128 * 4; // float [2 item][2 wg][128]
     static constexpr int OFF_BAR = OFF_DSUM + 2 * 2 * 128 * 4;
-    static constexpr int NBAR = 3 * 2 + 4 * 3 + 7 * 2 + 2;
+    static constexpr int NBAR = 3 * 2 + 4 * 4 + 3 * 3 + 4 * 2 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack for 1024-B alignment
     static_assert(OFF_BAR % 8 == 0, "barrier alignment");
     static_assert(SMEM <= 232448, "shared memory per CTA");
+    static_assert(NST <= 4 && NBUF <= 3, "barrier arrays");
 };
 
 // Inverse RoPE of one accumulator row held in TMEM (fp32, D columns), for a
@@ -315,8 +321,8 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
     float *sDsum = reinterpret_cast<float *>(smem + C::OFF_DSUM);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *stat_full = bars, *stat_ready = bars + 2, *stat_free = bars + 4;
-    uint64_t *b1_full = bars + 6, *b2_full = b1_full + 3, *st_ready = b2_full + 3, *st_free = st_ready + 3;
-    uint64_t *x_full = st_free + 3, *p_full = x_full + 2, *buf_free = p_full + 2, *acc_full = buf_free + 2;
+    uint64_t *b1_full = bars + 6, *b2_full = b1_full + 4, *st_ready = b2_full + 4, *st_free = st_ready + 4;
+    uint64_t *x_full = st_free + 4, *p_full = x_full + 3, *buf_free = p_full + 3, *acc_full = buf_free + 3;
     uint64_t *acc_free = acc_full + 2, *dsum_full = acc_free + 2, *dsum_free = dsum_full + 2;
     uint64_t *drain_x = dsum_free + 2, *drain_g = drain_x + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
@@ -332,15 +338,17 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             sm100::mbar_init(stat_full + s, 1);
             sm100::mbar_init(stat_ready + s, 128);
             sm100::mbar_init(stat_free + s, 1);
-            sm100::mbar_init(x_full + s, 1);
-            sm100::mbar_init(p_full + s, 128);
-            sm100::mbar_init(buf_free + s, 1);
             sm100::mbar_init(acc_full + s, 1);
             sm100::mbar_init(acc_free + s, 128);
             sm100::mbar_init(dsum_full + s, 256);
             sm100::mbar_init(dsum_free + s, 128);
         }
         for (int s = 0; s < 3; ++s) {
+            sm100::mbar_init(x_full + s, 1);
+            sm100::mbar_init(p_full + s, 128);
+            sm100::mbar_init(buf_free + s, 1);
+        }
+        for (int s = 0; s < 4; ++s) {
             sm100::mbar_init(b1_full + s, 1);
             sm100::mbar_init(b2_full + s, 1);
             sm100::mbar_init(st_ready + s, 128);
@@ -390,7 +398,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
     if (warp == BWD_TMA_WARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int stat_par[2] = {-1, -1}, st_par[3] = {-1, -1, -1};
+            int stat_par[2] = {-1, -1}, st_par[4] = {-1, -1, -1, -1};
             int ts = 0, k = 0;
             bool ok = true;
             for (int u = u_begin; ok && u < u_end; ++u, ++k) {
@@ -421,7 +429,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             // every issued copy must have landed before the CTA may exit
             for (int s = 0; s < 2; ++s)
                 if (stat_par[s] >= 0) mbar_wait_drain(stat_full + s, stat_par[s]);
-            for (int s = 0; s < 3; ++s)
+            for (int s = 0; s < 4; ++s)
                 if (st_par[s] >= 0) { mbar_wait_drain(b1_full + s, st_par[s]); mbar_wait_drain(b2_full + s, st_par[s]); }
         }
     } else if (is_prep) {
@@ -477,10 +485,12 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                         // buffer h is free again once its previous half-step's S / dP were
                         // consumed: by the element-wise pass (P, dS elsewhere) or, when
                         // P / dS overlay S / dP, by the gradient MMAs
-                        if (hs >= 2 && !sm100::mbar_wait(C::SEP_PD ? p_full + h : buf_free + h, ((hs >> 1) - 1) & 1,
+                        constexpr int NB = C::NBUF;
+                        const int bf = hs % NB;
+                        if (hs >= NB && !sm100::mbar_wait(C::SEP_PD ? p_full + bf : buf_free + bf, ((hs / NB) - 1) & 1,
                                                          abort_flag)) { ok = false; break; }
                         sm100::tc_fence_after();
-                        const uint32_t dx = tmem + h * 128;
+                        const uint32_t dx = tmem + bf * 128;
 #pragma unroll
                         for (int ks = 0; ks < D / 16; ++ks) {
                             const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
@@ -491,7 +501,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                             const uint32_t off = (ks / 4) * C::HALF_BYTES + (ks % 4) * 32;
                             sm100::umma_ss(dx + 64, dsc(a2 + off), dsc(b2 + h * 8192 + off), IDESC_X, ks > 0 ? 1u : 0u);
                         }
-                        sm100::umma_commit(x_full + h);
+                        sm100::umma_commit(x_full + bf);
                     }
                 }
                 if (ok) sm100::umma_commit(stat_free + sb);   // the item's stationary tiles are read
@@ -517,7 +527,9 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                     const int s = ts % NST;
                     const uint32_t b1 = C::OFF_B1 + s * C::TILE, b2 = C::OFF_B2 + s * C::TILE;
                     for (int h = 0; h < 2; ++h, ++hs) {
-                        if (!sm100::mbar_wait(p_full + h, (hs >> 1) & 1, abort_flag)) { ok = false; break; }
+                        constexpr int NB = C::NBUF;
+                        const int bf = hs % NB;
+                        if (!sm100::mbar_wait(p_full + bf, (hs / NB) & 1, abort_flag)) { ok = false; break; }
                         if (ROLE != BWD_ROLE_DSUM) {
                             const bool first = (t == 0 && h == 0);
                             if (first && k >= NACC && !sm100::mbar_wait(acc_free + ab, ((k / NACC) - 1) & 1, abort_flag)) {
@@ -525,8 +537,8 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                                 break;
                             }
                             sm100::tc_fence_after();
-                            const uint32_t pa = C::SEP_PD ? tmem + 256 + h * C::PD_COLS : tmem + h * 128;
-                            const uint32_t da = C::SEP_PD ? pa + (ROLE == BWD_ROLE_DKDV ? 32 : 0) : tmem + h * 128 + 64;
+                            const uint32_t pa = C::SEP_PD ? tmem + C::NBUF * 128 + bf * C::PD_COLS : tmem + bf * 128;
+                            const uint32_t da = C::SEP_PD ? pa + (ROLE == BWD_ROLE_DKDV ? 32 : 0) : tmem + bf * 128 + 64;
                             if (ROLE == BWD_ROLE_DKDV) {
 #pragma unroll
                                 for (int ks = 0; ks < 4; ++ks)    // dV += P^T dO
@@ -543,7 +555,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                                                    (first && ks == 0) ? 0u : 1u);
                             }
                         }
-                        sm100::umma_commit(buf_free + h);
+                        sm100::umma_commit(buf_free + bf);
                         if (h == 1) sm100::umma_commit(st_free + s);   // the step's streamed tiles are read
                         if (ROLE != BWD_ROLE_DSUM && h == 1 && t == it.T - 1) sm100::umma_commit(acc_full + ab);
                     }
@@ -665,17 +677,18 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                 }
                 // decisions to stop are taken by the whole warpgroup (it also meets at
                 // named barriers), so no warp waits at one that the others left
-                const bool ok = sm100::mbar_wait(x_full + w, ts & 1, abort_flag);
+                const int hsm = 2 * ts + w, bf = hsm % C::NBUF;        // this half-step and its buffer
+                const bool ok = sm100::mbar_wait(x_full + bf, (hsm / C::NBUF) & 1, abort_flag);
                 if (named_bar_or(2 + w, 128, !ok)) { good = false; break; }
                 sm100::tc_fence_after();
-                if (C::SEP_PD && ts >= 1) {
+                if (C::SEP_PD && hsm >= C::NBUF) {
                     // P / dS columns of this buffer: read by the previous half-step's gradient MMAs
-                    const bool okp = sm100::mbar_wait(buf_free + w, (ts - 1) & 1, abort_flag);
+                    const bool okp = sm100::mbar_wait(buf_free + bf, ((hsm / C::NBUF) - 1) & 1, abort_flag);
                     if (named_bar_or(2 + w, 128, !okp)) { good = false; break; }
                     sm100::tc_fence_after();
                 }
-                const uint32_t x_addr = tmem + lane_base + w * 128;
-                const uint32_t p_addr = C::SEP_PD ? tmem + lane_base + 256 + w * C::PD_COLS : x_addr;
+                const uint32_t x_addr = tmem + lane_base + bf * 128;
+                const uint32_t p_addr = C::SEP_PD ? tmem + lane_base + C::NBUF * 128 + bf * C::PD_COLS : x_addr;
                 const uint32_t ds_addr = C::SEP_PD ? p_addr + (ROLE == BWD_ROLE_DKDV ? 32 : 0) : x_addr + 64;
                 if (ROLE == BWD_ROLE_DSUM)
                     dsum += bwd_half_step<MODE, false, false, true>(x_addr, p_addr, ds_addr, xs, b0, bstep, m, lrow,
@@ -688,7 +701,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                                                            colL, colD);
                 sm100::tmem_wait_st();
                 sm100::tc_fence_before();
-                sm100::mbar_arrive(p_full + w);
+                sm100::mbar_arrive(p_full + bf);
                 if (has_pend) {
                     has_pend = false;
                     if (!epilogue(pend)) { good = false; break; }
