@@ -83,7 +83,8 @@ SWAT_API int swat_attn_fwd(const void *q, const void *k, const void *v, void *o,
                   int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
                   const float *slopes, float rope_base, int dtype, void *stream);
 
-/* Bytes of device workspace swat_attn_bwd needs for these sizes. */
+/* Bytes of device workspace swat_attn_bwd needs for these sizes: the softmax
+ * row terms D_i ([B,H,N] fp32) and, for bf16, RoPE-rotated copies of Q and K. */
 SWAT_API size_t swat_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int d, int dtype);
 
 /* Backward of swat_attn_fwd (derived by calculus from the [SWAT] equation;

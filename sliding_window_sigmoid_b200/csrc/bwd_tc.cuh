@@ -25,8 +25,8 @@
 //   warps 4-11 two activation warpgroups (one TMEM lane = one row per thread);
 //              the epilogue of item k runs in warpgroup k % 2, deferred until
 //              after its next half-step.
-//   warps 12-15 RoPE prep: rotate the stationary Q or K tile and each streamed
-//              K or Q tile in place in shared memory.
+//   warps 12-15 set-up only. Q and K arrive RoPE-rotated: a small kernel
+//              writes rotated copies into the workspace first.
 // TMEM columns: [128 h, 128 h + 64) S half, [128 h + 64, 128 h + 128) dP half
 // (their first 32 columns then hold bf16 P and dS), accumulators from 256.
 #pragma once
@@ -297,6 +297,51 @@ __device__ __forceinline__ float bwd_half_step(uint32_t x_addr, uint32_t p_addr,
 }
 
 // ===========================================================================
+// RoPE of Q or K rows into a copy, once per backward call: both backward
+// kernels then load rotated tiles directly. x, y: [B, N, Hx, D] bf16. CTA =
+// 128 positions of one (b, head); the angle of pair t at position n0 + r is
+// A_t + r theta_t, A_t = n0 theta_t reduced mod 2 pi in fp64, the sum reduced
+// again in fp32 before __sincosf (|error| ~ 1e-6 rad).
+// ===========================================================================
+template <int D>
+__global__ void __launch_bounds__(256)
+swat_rope_rows_kernel(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ y, int N, int Hx,
+                      double log2_base)
+{
+    __shared__ float sA[D / 2], sT[D / 2];
+    const int n0 = blockIdx.x * 128, hx = blockIdx.y, b = blockIdx.z;
+    if (threadIdx.x < D / 2) {
+        const double th = exp2(-2.0 * (double)threadIdx.x / (double)D * log2_base);
+        const double two_pi = 6.283185307179586476925286766559;
+        const double an = (double)n0 * th;
+        sA[threadIdx.x] = (float)(an - rint(an / two_pi) * two_pi);
+        sT[threadIdx.x] = (float)th;
+    }
+    __syncthreads();
+    const float two_pi = 6.2831853071795865f, inv_two_pi = 0.15915494309189534f;
+    constexpr int CH = D / 8;                      // 16-byte chunks per row (4 pairs each)
+    for (int idx = threadIdx.x; idx < 128 * CH; idx += blockDim.x) {
+        const int r = idx / CH, c = idx % CH, n = n0 + r;
+        if (n >= N) break;
+        const size_t off = (((size_t)b * N + n) * Hx + hx) * D + 8 * c;
+        const uint4 in = *reinterpret_cast<const uint4 *>(x + off);
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const int t = 4 * c + p;
+            float ang = fmaf((float)r, sT[t], sA[t]);
+            ang = fmaf(-rintf(ang * inv_two_pi), two_pi, ang);
+            float sn, cs;
+            __sincosf(ang, &sn, &cs);
+            const float x0 = sm100::bf16lo(w[p]), x1 = sm100::bf16hi(w[p]);
+            o[p] = sm100::pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+        }
+        *reinterpret_cast<uint4 *>(y + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// ===========================================================================
 // The persistent backward kernel.
 // tm_a1/tm_a2: stationary tensors (DQ, DSUM: Q, dO; DKDV: K, V);
 // tm_b1/tm_b2: streamed tensors (DQ, DSUM: K, V; DKDV: Q, dO). Tiles a1 and
@@ -313,7 +358,6 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA1 = smem + C::OFF_A1, *sA2 = smem + C::OFF_A2, *sB1 = smem + C::OFF_B1, *sB2 = smem + C::OFF_B2;
-    float2 *sRot = reinterpret_cast<float2 *>(smem + C::OFF_ROT);
     double *sTh = reinterpret_cast<double *>(smem + C::OFF_TH);
     float *sThf = reinterpret_cast<float *>(smem + C::OFF_THF);
     float *sA0 = reinterpret_cast<float *>(smem + C::OFF_A0);
@@ -371,24 +415,10 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
     }
     const bool is_prep = warp >= BWD_PREP_WARP0;
     const int ptid = threadIdx.x - 32 * BWD_PREP_WARP0;
-    RotThread rot;
-    if (is_prep) {
-        if (ptid < D / 2) {
-            const double th = exp2(-2.0 * (double)ptid / (double)D * a.log2_base);
-            sTh[ptid] = th;
-            sThf[ptid] = (float)th;
-        }
-        sm100::named_bar_sync(FWD_PREP_BAR, 128);
-        if (a.use_rope) {
-            constexpr int CPR = D / 8, RS = 128 / CPR;
-            const int c = ptid % CPR, r0 = ptid / CPR;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const double th = sTh[4 * c + q];
-                const float2 w0 = rope_cs((double)r0 * th), stp = rope_cs((double)RS * th);
-                rot.w0c[q] = w0.x; rot.w0s[q] = w0.y; rot.stc[q] = stp.x; rot.sts[q] = stp.y;
-            }
-        }
+    if (is_prep && ptid < D / 2) {   // RoPE frequencies for the epilogue's inverse rotation
+        const double th = exp2(-2.0 * (double)ptid / (double)D * a.log2_base);
+        sTh[ptid] = th;
+        sThf[ptid] = (float)th;
     }
     sm100::tc_fence_before();
     __syncthreads();
@@ -432,36 +462,6 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             for (int s = 0; s < 4; ++s)
                 if (st_par[s] >= 0) { mbar_wait_drain(b1_full + s, st_par[s]); mbar_wait_drain(b2_full + s, st_par[s]); }
         }
-    } else if (is_prep) {
-        // ------------------------------------------------------------ RoPE prep
-        int ebuf = 0;
-        auto make_bases = [&](int pos0) {
-            ebuf ^= 1;
-            if (a.use_rope && ptid < D / 2) sRot[ebuf * (D / 2) + ptid] = rope_cs((double)pos0 * sTh[ptid]);
-        };
-        int ts = 0, k = 0;
-        bool ok = true;
-        for (int u = u_begin; ok && u < u_end; ++u, ++k) {
-            const BwdItem it = bwd_item<ROLE>(a, u);
-            const int sb = k % NSTAT;
-            make_bases(it.row0);
-            bool w_ok = sm100::mbar_wait(stat_full + sb, (k / NSTAT) & 1, abort_flag);
-            if (named_bar_or(FWD_PREP_BAR, 128, !w_ok || *abort_flag)) break;
-            if (a.use_rope) rope_rotate_tile<D>(sA1 + sb * C::TILE, sRot + ebuf * (D / 2), rot, ptid);
-            sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(stat_ready + sb);
-            for (int t = 0; t < it.T; ++t, ++ts) {
-                const int s = ts % NST;
-                int head, pos0;
-                bwd_stream<ROLE>(it, G, t, head, pos0);
-                make_bases(pos0);
-                w_ok = sm100::mbar_wait(b1_full + s, (ts / NST) & 1, abort_flag);
-                if (named_bar_or(FWD_PREP_BAR, 128, !w_ok || *abort_flag)) { ok = false; break; }
-                if (a.use_rope) rope_rotate_tile<D>(sB1 + s * C::TILE, sRot + ebuf * (D / 2), rot, ptid);
-                sm100::fence_proxy_async_smem();
-                sm100::mbar_arrive(st_ready + s);
-            }
-        }
     } else if (warp == BWD_X_WARP) {
         // ------------------------------------------------------------ X MMAs: S half and dP half
         if (lane == 0) {
@@ -474,11 +474,11 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             for (int u = u_begin; ok && u < u_end; ++u, ++k) {
                 const BwdItem it = bwd_item<ROLE>(a, u);
                 const int sb = k % NSTAT;
-                if (!sm100::mbar_wait(stat_ready + sb, (k / NSTAT) & 1, abort_flag)) break;
+                if (!sm100::mbar_wait(stat_full + sb, (k / NSTAT) & 1, abort_flag)) break;
                 const uint32_t a1 = C::OFF_A1 + sb * C::TILE, a2 = C::OFF_A2 + sb * C::TILE;
                 for (int t = 0; ok && t < it.T; ++t, ++ts) {
                     const int s = ts % NST;
-                    if (!sm100::mbar_wait(st_ready + s, (ts / NST) & 1, abort_flag) ||
+                    if (!sm100::mbar_wait(b1_full + s, (ts / NST) & 1, abort_flag) ||
                         !sm100::mbar_wait(b2_full + s, (ts / NST) & 1, abort_flag)) { ok = false; break; }
                     const uint32_t b1 = C::OFF_B1 + s * C::TILE, b2 = C::OFF_B2 + s * C::TILE;
                     for (int h = 0; h < 2; ++h, ++hs) {
@@ -565,7 +565,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             mbar_wait_drain(drain_g, 0);
         }
         __syncwarp();
-    } else if (warp >= BWD_ACT_WARP0) {
+    } else if (warp >= BWD_ACT_WARP0 && warp < BWD_PREP_WARP0) {
         // ------------------------------------------------------------ activation + epilogue
         const int w = (warp - BWD_ACT_WARP0) / 4;                 // warpgroup = half of every step
         const int r = 32 * (warp % 4) + lane;                     // stationary row (= TMEM lane)
@@ -754,14 +754,30 @@ inline bool launch_bwd_role(const BwdArgs &a, const CUtensorMap &tq, const CUten
     return true;
 }
 
+inline size_t bwd_align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
 template <int D, int MODE>
-inline int launch_bwd_tc_t(const BwdArgs &a, cudaStream_t stream)
+inline int launch_bwd_tc_t(const BwdArgs &a, void *extra_ws, cudaStream_t stream)
 {
+    int n = 0;
+    const void *qr = a.q, *kr = a.k;
+    if (a.use_rope) {   // rotated copies of Q and K in the workspace
+        __nv_bfloat16 *wq = reinterpret_cast<__nv_bfloat16 *>(extra_ws);
+        __nv_bfloat16 *wk = reinterpret_cast<__nv_bfloat16 *>(
+            reinterpret_cast<char *>(extra_ws) + bwd_align256((size_t)a.B * a.N * a.H * D * 2));
+        const unsigned nqt = (unsigned)((a.N + 127) / 128);
+        swat_rope_rows_kernel<D><<<dim3(nqt, a.H, a.B), 256, 0, stream>>>(
+            reinterpret_cast<const __nv_bfloat16 *>(a.q), wq, a.N, a.H, a.log2_base);
+        swat_rope_rows_kernel<D><<<dim3(nqt, a.Hkv, a.B), 256, 0, stream>>>(
+            reinterpret_cast<const __nv_bfloat16 *>(a.k), wk, a.N, a.Hkv, a.log2_base);
+        qr = wq;
+        kr = wk;
+        n += 2;
+    }
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_tmap_bshd(&tq, a.q, a.B, a.N, a.H, D) || !make_tmap_bshd(&tk, a.k, a.B, a.N, a.Hkv, D) ||
+    if (!make_tmap_bshd(&tq, qr, a.B, a.N, a.H, D) || !make_tmap_bshd(&tk, kr, a.B, a.N, a.Hkv, D) ||
         !make_tmap_bshd(&tv, a.v, a.B, a.N, a.Hkv, D) || !make_tmap_bshd(&tdo, a.dout, a.B, a.N, a.H, D))
         return -1;
-    int n = 0;
     if (MODE == SWAT_MODE_SOFTMAX_) {
         if (!launch_bwd_role<D, MODE, BWD_ROLE_DSUM>(a, tq, tk, tv, tdo, stream)) return -1;
         ++n;
@@ -771,22 +787,21 @@ inline int launch_bwd_tc_t(const BwdArgs &a, cudaStream_t stream)
     return n + 2;
 }
 
+// Workspace after the softmax D_i: RoPE-rotated copies of Q and K (bf16).
 inline size_t tc_bwd_extra_workspace(int B, int H, int Hkv, int N, int d)
 {
-    (void)B; (void)H; (void)Hkv; (void)N; (void)d;
-    return 0;
+    return bwd_align256((size_t)B * N * H * d * 2) + bwd_align256((size_t)B * N * Hkv * d * 2);
 }
 
 // Returns the number of kernels launched, or -1 on a launch-configuration error.
 inline int launch_bwd_tc(const BwdArgs &a, void *extra_ws, cudaStream_t stream)
 {
-    (void)extra_ws;
     if (a.d == 64)
-        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<64, SWAT_MODE_SIGMOID_>(a, stream)
-                                            : launch_bwd_tc_t<64, SWAT_MODE_SOFTMAX_>(a, stream);
+        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<64, SWAT_MODE_SIGMOID_>(a, extra_ws, stream)
+                                            : launch_bwd_tc_t<64, SWAT_MODE_SOFTMAX_>(a, extra_ws, stream);
     if (a.d == 128)
-        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<128, SWAT_MODE_SIGMOID_>(a, stream)
-                                            : launch_bwd_tc_t<128, SWAT_MODE_SOFTMAX_>(a, stream);
+        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<128, SWAT_MODE_SIGMOID_>(a, extra_ws, stream)
+                                            : launch_bwd_tc_t<128, SWAT_MODE_SOFTMAX_>(a, extra_ws, stream);
     return -1;
 }
 
