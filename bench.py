@@ -252,10 +252,12 @@ def run_swat(args):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(16, binding.bwd_workspace_bytes(B, H, Hkv, N, d)), dtype=torch.uint8,
                      device=dev)
+    fws = torch.empty(max(16, binding.fwd_workspace_bytes(B, H, Hkv, N, d)), dtype=torch.uint8,
+                      device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        binding.attn_fwd(q, k, v, out=o, **kw)
+        binding.attn_fwd(q, k, v, out=o, workspace=fws, **kw)
         binding.attn_bwd(q, k, v, o, None, do, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
 
     for _ in range(args.warmup):
@@ -277,7 +279,7 @@ def run_swat(args):
     start.record(stream)
     for i in range(args.steps):
         evs[i][0].record(stream)
-        binding.attn_fwd(q, k, v, out=o, **kw)
+        binding.attn_fwd(q, k, v, out=o, workspace=fws, **kw)
         evs[i][1].record(stream)
         binding.attn_bwd(q, k, v, o, None, do, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
         evs[i][2].record(stream)
@@ -310,12 +312,12 @@ def run_swat(args):
     # ---- end to end through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
-        e2e = bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, kw)
+        e2e = bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, fws, kw)
 
     # ---- ring-buffer decode (batch 64, 32/8 heads, d 128, window 4096) ----
     decode = {}
     if not args.no_decode:
-        del q, k, v, do, o, dq, dk, dv, ws
+        del q, k, v, do, o, dq, dk, dv, ws, fws
         torch.cuda.empty_cache()
         decode = bench_decode(args, dev, world, rank, peaks, peak_src)
 
@@ -326,7 +328,7 @@ def run_swat(args):
                 launches, fwd_tf, bwd_tf, decode)
 
 
-def bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, kw):
+def bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, fws, kw):
     """Same step through the public API with host buffers: every step copies
     Q, K, V, dO from pinned host memory and reads O, dQ, dK, dV back."""
     import torch
@@ -341,7 +343,7 @@ def bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, k
         dk_in.copy_(hk, non_blocking=True)
         dv_in.copy_(hv, non_blocking=True)
         ddo_in.copy_(hdo, non_blocking=True)
-        binding.attn_fwd(dq_in, dk_in, dv_in, out=o, **kw)
+        binding.attn_fwd(dq_in, dk_in, dv_in, out=o, workspace=fws, **kw)
         binding.attn_bwd(dq_in, dk_in, dv_in, o, None, ddo_in, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
         ho.copy_(o, non_blocking=True)
         hdq.copy_(dq, non_blocking=True)

@@ -83,6 +83,25 @@ SWAT_API int swat_attn_fwd(const void *q, const void *k, const void *v, void *o,
                   int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
                   const float *slopes, float rope_base, int dtype, void *stream);
 
+/* Bytes of device workspace swat_attn_fwd_ws needs: RoPE-rotated copies of Q
+ * and K (bf16 [B,N,H,d] and [B,N,Hkv,d], each padded to 256 bytes) for the
+ * bf16 path; 0 for fp32 or invalid sizes. */
+SWAT_API size_t swat_attn_fwd_workspace_bytes(int B, int H, int Hkv, int N, int d, int dtype);
+
+/* swat_attn_fwd with a workspace: same operation, arguments, layouts and
+ * results. With bf16 and RoPE on, Q and K are first rotated into the
+ * workspace by a small element-wise kernel and the attention kernel loads
+ * rotated tiles, instead of rotating each staged tile in shared memory.
+ *   workspace: swat_attn_fwd_workspace_bytes() bytes of device memory,
+ *              16-byte aligned (required for bf16; ignored for fp32); its
+ *              contents on entry do not matter, and it may be reused as
+ *              soon as the call's work on `stream` has finished.
+ * Returns SWAT_ERR_INVALID_ARG for a missing or misaligned bf16 workspace;
+ * otherwise as swat_attn_fwd. */
+SWAT_API int swat_attn_fwd_ws(const void *q, const void *k, const void *v, void *o, float *lse, void *workspace,
+                  int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
+                  const float *slopes, float rope_base, int dtype, void *stream);
+
 /* Bytes of device workspace swat_attn_bwd needs for these sizes: the softmax
  * row terms D_i ([B,H,N] fp32) and, for bf16, RoPE-rotated copies of Q and K. */
 SWAT_API size_t swat_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int d, int dtype);

@@ -26,7 +26,7 @@ _STATUS = {0: "SWAT_OK", -1: "SWAT_ERR_INVALID_ARG", -2: "SWAT_ERR_UNSUPPORTED",
 SCRATCH_LIMIT = -5
 NOALLOC_SCRATCH_BYTES = 16 << 20   # SWA_DECODE_NOALLOC_SCRATCH_BYTES
 
-EXPORTED = ["swat_attn_fwd", "swat_attn_bwd_workspace_bytes", "swat_attn_bwd", "swa_cache_fill",
+EXPORTED = ["swat_attn_fwd", "swat_attn_fwd_workspace_bytes", "swat_attn_fwd_ws", "swat_attn_bwd_workspace_bytes", "swat_attn_bwd", "swa_cache_fill",
             "swa_decode_step", "swa_decode_workspace_bytes", "swa_decode_step_noalloc", "swat_status_string",
             "swat_get_device_status", "swat_launch_count"]
 
@@ -52,6 +52,10 @@ def lib() -> ctypes.CDLL:
     P, I, F, LL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong, ctypes.c_size_t
     L.swat_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, P, F, I, P]
     L.swat_attn_fwd.restype = I
+    L.swat_attn_fwd_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    L.swat_attn_fwd_workspace_bytes.restype = SZ
+    L.swat_attn_fwd_ws.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, F, I, P]
+    L.swat_attn_fwd_ws.restype = I
     L.swat_attn_bwd_workspace_bytes.argtypes = [I, I, I, I, I, I]
     L.swat_attn_bwd_workspace_bytes.restype = SZ
     L.swat_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, F, I, P]
@@ -120,10 +124,18 @@ def _slopes(slopes, H, device):
     return s
 
 
+def fwd_workspace_bytes(B, H, Hkv, N, d, dtype=BF16) -> int:
+    return int(lib().swat_attn_fwd_workspace_bytes(B, H, Hkv, N, d, dtype))
+
+
 def attn_fwd(q, k, v, *, window: int, n_sink: int = 0, mode: int = MODE_SIGMOID, slopes=None,
-             rope_base: float = 10000.0, out=None, lse=None, stream=None):
+             rope_base: float = 10000.0, out=None, lse=None, workspace=None, stream=None):
     """SWAT forward. q [B,N,H,d], k/v [B,N,Hkv,d] (bf16 or fp32, CUDA).
-    Returns (o [B,N,H,d], lse [B,H,N] fp32 or None in sigmoid mode)."""
+    Returns (o [B,N,H,d], lse [B,H,N] fp32 or None in sigmoid mode).
+
+    workspace: None allocates one and calls swat_attn_fwd_ws (rotated Q/K
+    copies); a uint8 CUDA tensor of fwd_workspace_bytes() is used as given;
+    False calls swat_attn_fwd (tiles rotated in shared memory)."""
     B, N, H, d = q.shape
     Hkv = k.shape[2]
     dev = q.device
@@ -134,10 +146,17 @@ def attn_fwd(q, k, v, *, window: int, n_sink: int = 0, mode: int = MODE_SIGMOID,
     if mode == MODE_SOFTMAX and lse is None:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
     sl = _slopes(slopes, H, dev)
-    st = lib().swat_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, d,
-                             window, n_sink, mode, _ptr(sl), float(rope_base), _dtype_code(q),
-                             _stream(stream))
-    _check("swat_attn_fwd", st)
+    args = (B, H, Hkv, N, d, window, n_sink, mode, _ptr(sl), float(rope_base), _dtype_code(q),
+            _stream(stream))
+    if workspace is False:
+        st = lib().swat_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), *args)
+        _check("swat_attn_fwd", st)
+        return out, lse
+    if workspace is None:
+        nbytes = fwd_workspace_bytes(B, H, Hkv, N, d, _dtype_code(q))
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    st = lib().swat_attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(workspace), *args)
+    _check("swat_attn_fwd_ws", st)
     return out, lse
 
 

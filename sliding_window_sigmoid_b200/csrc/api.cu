@@ -78,7 +78,11 @@ int swat_get_device_status(void *stream)
     return h;
 }
 
-int swat_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+}  // extern "C"
+
+namespace {
+// The forward with an optional workspace for RoPE-rotated copies of Q and K.
+int attn_fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, void *workspace,
                   int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
                   const float *slopes, float rope_base, int dtype, void *stream)
 {
@@ -97,7 +101,7 @@ int swat_attn_fwd(const void *q, const void *k, const void *v, void *o, float *l
         a.B = B; a.H = H; a.Hkv = Hkv; a.N = N; a.d = d; a.window = window; a.n_sink = n_sink;
         a.mode = mode; a.use_rope = rope_base > 0.f; a.log2_base = log2_base_of(rope_base);
         a.scale = (float)(1.0 / sqrt((double)d));
-        int n = swat::launch_fwd_tc(a, S(stream));
+        int n = swat::launch_fwd_tc(a, workspace, S(stream));
         if (n < 0) return SWAT_ERR_CUDA;
         return after_launch(n);
     }
@@ -111,6 +115,32 @@ int swat_attn_fwd(const void *q, const void *k, const void *v, void *o, float *l
     cudaFuncSetAttribute(swat::swat_fwd_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     swat::swat_fwd_simt_kernel<float><<<grid, swat::SIMT_THREADS, smem, S(stream)>>>(a);
     return after_launch(1);
+}
+}  // namespace
+
+extern "C" {
+
+int swat_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
+                  const float *slopes, float rope_base, int dtype, void *stream)
+{
+    return attn_fwd_impl(q, k, v, o, lse, nullptr, B, H, Hkv, N, d, window, n_sink, mode, slopes, rope_base,
+                         dtype, stream);
+}
+
+size_t swat_attn_fwd_workspace_bytes(int B, int H, int Hkv, int N, int d, int dtype)
+{
+    if (B < 1 || H < 1 || Hkv < 1 || N < 1 || d < 2 || dtype != SWAT_BF16) return 0;
+    return swat::rope_copies_bytes(B, H, Hkv, N, d);
+}
+
+int swat_attn_fwd_ws(const void *q, const void *k, const void *v, void *o, float *lse, void *workspace,
+                     int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
+                     const float *slopes, float rope_base, int dtype, void *stream)
+{
+    if (dtype == SWAT_BF16 && (!workspace || !aligned16(workspace))) return SWAT_ERR_INVALID_ARG;
+    return attn_fwd_impl(q, k, v, o, lse, dtype == SWAT_BF16 ? workspace : nullptr, B, H, Hkv, N, d, window,
+                         n_sink, mode, slopes, rope_base, dtype, stream);
 }
 
 size_t swat_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int d, int dtype)

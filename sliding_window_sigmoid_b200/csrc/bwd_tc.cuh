@@ -31,6 +31,7 @@
 // (their first 32 columns then hold bf16 P and dS), accumulators from 256.
 #pragma once
 #include "fwd_tc.cuh"
+#include "rope_rows.cuh"
 
 namespace swat {
 
@@ -294,51 +295,6 @@ __device__ __forceinline__ float bwd_half_step(uint32_t x_addr, uint32_t p_addr,
         if (WRITE_DS) sm100::tmem_st16(ds_addr + 16 * cc, gk);
     }
     return dsum;
-}
-
-// ===========================================================================
-// RoPE of Q or K rows into a copy, once per backward call: both backward
-// kernels then load rotated tiles directly. x, y: [B, N, Hx, D] bf16. CTA =
-// 128 positions of one (b, head); the angle of pair t at position n0 + r is
-// A_t + r theta_t, A_t = n0 theta_t reduced mod 2 pi in fp64, the sum reduced
-// again in fp32 before __sincosf (|error| ~ 1e-6 rad).
-// ===========================================================================
-template <int D>
-__global__ void __launch_bounds__(256)
-swat_rope_rows_kernel(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ y, int N, int Hx,
-                      double log2_base)
-{
-    __shared__ float sA[D / 2], sT[D / 2];
-    const int n0 = blockIdx.x * 128, hx = blockIdx.y, b = blockIdx.z;
-    if (threadIdx.x < D / 2) {
-        const double th = exp2(-2.0 * (double)threadIdx.x / (double)D * log2_base);
-        const double two_pi = 6.283185307179586476925286766559;
-        const double an = (double)n0 * th;
-        sA[threadIdx.x] = (float)(an - rint(an / two_pi) * two_pi);
-        sT[threadIdx.x] = (float)th;
-    }
-    __syncthreads();
-    const float two_pi = 6.2831853071795865f, inv_two_pi = 0.15915494309189534f;
-    constexpr int CH = D / 8;                      // 16-byte chunks per row (4 pairs each)
-    for (int idx = threadIdx.x; idx < 128 * CH; idx += blockDim.x) {
-        const int r = idx / CH, c = idx % CH, n = n0 + r;
-        if (n >= N) break;
-        const size_t off = (((size_t)b * N + n) * Hx + hx) * D + 8 * c;
-        const uint4 in = *reinterpret_cast<const uint4 *>(x + off);
-        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int t = 4 * c + p;
-            float ang = fmaf((float)r, sT[t], sA[t]);
-            ang = fmaf(-rintf(ang * inv_two_pi), two_pi, ang);
-            float sn, cs;
-            __sincosf(ang, &sn, &cs);
-            const float x0 = sm100::bf16lo(w[p]), x1 = sm100::bf16hi(w[p]);
-            o[p] = sm100::pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
-        }
-        *reinterpret_cast<uint4 *>(y + off) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
 }
 
 // ===========================================================================
@@ -754,26 +710,13 @@ inline bool launch_bwd_role(const BwdArgs &a, const CUtensorMap &tq, const CUten
     return true;
 }
 
-inline size_t bwd_align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
 template <int D, int MODE>
 inline int launch_bwd_tc_t(const BwdArgs &a, void *extra_ws, cudaStream_t stream)
 {
     int n = 0;
     const void *qr = a.q, *kr = a.k;
-    if (a.use_rope) {   // rotated copies of Q and K in the workspace
-        __nv_bfloat16 *wq = reinterpret_cast<__nv_bfloat16 *>(extra_ws);
-        __nv_bfloat16 *wk = reinterpret_cast<__nv_bfloat16 *>(
-            reinterpret_cast<char *>(extra_ws) + bwd_align256((size_t)a.B * a.N * a.H * D * 2));
-        const unsigned nqt = (unsigned)((a.N + 127) / 128);
-        swat_rope_rows_kernel<D><<<dim3(nqt, a.H, a.B), 256, 0, stream>>>(
-            reinterpret_cast<const __nv_bfloat16 *>(a.q), wq, a.N, a.H, a.log2_base);
-        swat_rope_rows_kernel<D><<<dim3(nqt, a.Hkv, a.B), 256, 0, stream>>>(
-            reinterpret_cast<const __nv_bfloat16 *>(a.k), wk, a.N, a.Hkv, a.log2_base);
-        qr = wq;
-        kr = wk;
-        n += 2;
-    }
+    if (a.use_rope)   // rotated copies of Q and K in the workspace
+        n += launch_rope_copies<D>(a.q, a.k, extra_ws, a.B, a.H, a.Hkv, a.N, a.log2_base, stream, &qr, &kr);
     CUtensorMap tq, tk, tv, tdo;
     if (!make_tmap_bshd(&tq, qr, a.B, a.N, a.H, D) || !make_tmap_bshd(&tk, kr, a.B, a.N, a.Hkv, D) ||
         !make_tmap_bshd(&tv, a.v, a.B, a.N, a.Hkv, D) || !make_tmap_bshd(&tdo, a.dout, a.B, a.N, a.H, D))
@@ -790,7 +733,7 @@ inline int launch_bwd_tc_t(const BwdArgs &a, void *extra_ws, cudaStream_t stream
 // Workspace after the softmax D_i: RoPE-rotated copies of Q and K (bf16).
 inline size_t tc_bwd_extra_workspace(int B, int H, int Hkv, int N, int d)
 {
-    return bwd_align256((size_t)B * N * H * d * 2) + bwd_align256((size_t)B * N * Hkv * d * 2);
+    return rope_copies_bytes(B, H, Hkv, N, d);
 }
 
 // Returns the number of kernels launched, or -1 on a launch-configuration error.

@@ -31,6 +31,7 @@
 #include "sm100.cuh"
 #include "fwd_simt.cuh"
 #include "bwd_simt.cuh"
+#include "rope_rows.cuh"
 
 namespace swat {
 
@@ -534,7 +535,9 @@ __device__ __forceinline__ float act_softmax_p(uint32_t s_addr, float sc2, float
     return lsum;
 }
 
-template <int D, int MODE>
+// PRE: Q and K arrive RoPE-rotated (copies in a workspace): the prep
+// warpgroup idles and the S MMAs wait for the TMA copies only.
+template <int D, int MODE, bool PRE>
 __global__ void __launch_bounds__(FwdRoles<MODE>::THREADS, 1)
 swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs a)
@@ -608,7 +611,7 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int ptid = threadIdx.x - 32 * FWD_PREP_WARP0;   // 0..127 inside the prep group
     const bool is_prep = warp >= FWD_PREP_WARP0 && warp < FWD_PREP_WARP0 + 4;
     RotThread rot;
-    if (is_prep && a.use_rope) {
+    if (!PRE && is_prep && a.use_rope) {
         if (ptid < D / 2) sTh[ptid] = exp2(-2.0 * (double)ptid / (double)D * a.log2_base);
         sm100::named_bar_sync(FWD_PREP_BAR, 128);
         constexpr int CPR = D / 8, RS = 128 / CPR;
@@ -694,7 +697,7 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     mbar_wait_drain(v_full + s, last_par[s]);
                 }
         }
-    } else if (is_prep) {
+    } else if (is_prep && !PRE) {
         // ------------------------------------------------------------ RoPE prep
         int ebuf = 0;
         auto make_bases = [&](int pos0) {
@@ -737,8 +740,11 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int idx = 0;; ++idx) {
                 if (!rec_read(sRec, rec_full, rec_free, NREC, RGRP, idx, abort_flag, r) || r.step < 0) break;
                 const int qs = r.k & 1, sb = r.step % NSB, slot = (int)(r.fl >> 8);
-                if ((r.fl & REC_FIRST) && !sm100::mbar_wait(q_ready + qs, (r.k >> 1) & 1, abort_flag)) break;
-                if ((r.fl & REC_NEW) && !sm100::mbar_wait(k_ready + slot, (r.fl & REC_PAR) ? 1 : 0, abort_flag)) break;
+                if ((r.fl & REC_FIRST) && !sm100::mbar_wait((PRE ? q_full : q_ready) + qs, (r.k >> 1) & 1, abort_flag))
+                    break;
+                if ((r.fl & REC_NEW) &&
+                    !sm100::mbar_wait((PRE ? k_full : k_ready) + slot, (r.fl & REC_PAR) ? 1 : 0, abort_flag))
+                    break;
                 if (r.step >= NSB && !sm100::mbar_wait(pv_done + sb, ((r.step / NSB) - 1) & 1, abort_flag)) break;
                 sm100::tc_fence_after();
                 const uint32_t lq = lo_q + (uint32_t)qs * TILE16, lk = lo_k + (uint32_t)slot * TILE16;
@@ -782,7 +788,7 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_wait_drain(drain_pv, 0);
         }
         __syncwarp();
-    } else if (warp >= FWD_ACT_WARP0) {
+    } else if (warp >= FWD_ACT_WARP0 && warp < FWD_PREP_WARP0) {
         // ------------------------------------------------------------ activation + epilogue
         // The epilogue of an item (O: TMEM -> bf16 global rows) is deferred to
         // after this warpgroup's next tile: by then the item's last P.V has
@@ -935,31 +941,37 @@ inline int num_sms()
 }
 
 template <int D, int MODE>
-inline int launch_fwd_tc_t(const FwdArgs &a, cudaStream_t stream)
+inline int launch_fwd_tc_t(const FwdArgs &a, void *ws, cudaStream_t stream)
 {
     using C = FwdTcCfg<D>;
+    int n = 0;
+    const void *qr = a.q, *kr = a.k;
+    const bool pre = ws != nullptr && a.use_rope;
+    if (pre) n += launch_rope_copies<D>(a.q, a.k, ws, a.B, a.H, a.Hkv, a.N, a.log2_base, stream, &qr, &kr);
     CUtensorMap tq, tk, tv;
-    if (!make_tmap_bshd(&tq, a.q, a.B, a.N, a.H, D) || !make_tmap_bshd(&tk, a.k, a.B, a.N, a.Hkv, D) ||
+    if (!make_tmap_bshd(&tq, qr, a.B, a.N, a.H, D) || !make_tmap_bshd(&tk, kr, a.B, a.N, a.Hkv, D) ||
         !make_tmap_bshd(&tv, a.v, a.B, a.N, a.Hkv, D))
         return -1;
-    auto kern = swat_fwd_tc_kernel<D, MODE>;
+    auto kern = pre ? swat_fwd_tc_kernel<D, MODE, true> : swat_fwd_tc_kernel<D, MODE, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return -1;
     const long long items = (long long)a.B * a.H * ((a.N + 127) / 128);
     if (items >= (1LL << 31)) return -1;   // the schedule decodes item indices in 32 bits
     const int grid = (int)std::min<long long>(items, (long long)num_sms());
     kern<<<grid, FwdRoles<MODE>::THREADS, C::SMEM, stream>>>(tq, tk, tv, a);
-    return 1;
+    return n + 1;
 }
 
-// Returns the number of kernels launched, or -1 on a launch-configuration error.
-inline int launch_fwd_tc(const TcFwdArgs &a, cudaStream_t stream)
+// ws: NULL (rotate Q and K tiles in shared memory) or rope_copies_bytes()
+// of device memory for rotated copies. Returns the number of kernels
+// launched, or -1 on a launch-configuration error.
+inline int launch_fwd_tc(const TcFwdArgs &a, void *ws, cudaStream_t stream)
 {
     if (a.d == 64)
-        return a.mode == SWAT_MODE_SIGMOID_ ? launch_fwd_tc_t<64, SWAT_MODE_SIGMOID_>(a, stream)
-                                            : launch_fwd_tc_t<64, SWAT_MODE_SOFTMAX_>(a, stream);
+        return a.mode == SWAT_MODE_SIGMOID_ ? launch_fwd_tc_t<64, SWAT_MODE_SIGMOID_>(a, ws, stream)
+                                            : launch_fwd_tc_t<64, SWAT_MODE_SOFTMAX_>(a, ws, stream);
     if (a.d == 128)
-        return a.mode == SWAT_MODE_SIGMOID_ ? launch_fwd_tc_t<128, SWAT_MODE_SIGMOID_>(a, stream)
-                                            : launch_fwd_tc_t<128, SWAT_MODE_SOFTMAX_>(a, stream);
+        return a.mode == SWAT_MODE_SIGMOID_ ? launch_fwd_tc_t<128, SWAT_MODE_SIGMOID_>(a, ws, stream)
+                                            : launch_fwd_tc_t<128, SWAT_MODE_SOFTMAX_>(a, ws, stream);
     return -1;
 }
 

@@ -104,7 +104,10 @@ def test_index_probe_bit_exact(dtype, N, w, s):
     (1, 1, 4, 1, 450, 64, 30, 64, 1e4, None),           # many sinks
     (0, 1, 4, 2, 300, 128, 50, 7, 1e4, "balanced"),     # sinks in sigmoid mode
 ])
-def test_bf16_matches_oracle(mode, B, H, Hkv, N, d, w, s, base, slopes):
+@pytest.mark.parametrize("ws", ["rotated copies", "in-kernel rotation"])
+def test_bf16_matches_oracle(mode, B, H, Hkv, N, d, w, s, base, slopes, ws):
+    """Both entry points: swat_attn_fwd_ws (rotated Q/K copies in a workspace)
+    and swat_attn_fwd (tiles rotated in shared memory)."""
     scale = 1.0 / np.sqrt(d) if mode == 0 else 1.0
     q, k, v = inputs.qkv(B, N, H, Hkv, d, seed=2, scale=scale, dtype=torch.bfloat16)
     sl = None
@@ -112,7 +115,8 @@ def test_bf16_matches_oracle(mode, B, H, Hkv, N, d, w, s, base, slopes):
         sl = inputs.balanced_alibi_slopes(H)
     elif slopes == "geometric":
         sl = inputs.geometric_alibi_slopes(H)
-    o, lse = _run_fwd(q, k, v, window=w, n_sink=s, mode=mode, slopes=sl, rope_base=base)
+    o, lse = _run_fwd(q, k, v, window=w, n_sink=s, mode=mode, slopes=sl, rope_base=base,
+                      workspace=None if ws == "rotated copies" else False)
     ref, lref = oracle.swat_fwd(q.float().numpy(), k.float().numpy(), v.float().numpy(), window=w,
                                 n_sink=s, mode=mode, slopes=None if sl is None else sl.numpy(),
                                 rope_base=base)
