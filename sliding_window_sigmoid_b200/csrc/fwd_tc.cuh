@@ -69,16 +69,20 @@ struct FwdTcCfg {
 // walks the schedule ahead of them (StepRec ring); warp 3 issues P.V.
 // Activation warpgroups start at warp 4 so that warp w owns TMEM lanes
 // 32 (w % 4) .. 32 (w % 4) + 31.
-template <int MODE>
+template <int D, int MODE, bool PRE>
 struct FwdRoles {
-    static constexpr int ACT_WG = (MODE == SWAT_MODE_SIGMOID_) ? 2 : 1;
+    // sigmoid: 2 activation warpgroups; 3 when Q and K arrive rotated (the
+    // prep warps are then free) and there are 3 S buffers (d 64), so that
+    // each warpgroup owns one buffer and waits on its barriers in order (an
+    // mbarrier parity wait must not run a phase ahead); softmax: 1
+    static constexpr int ACT_WG = (MODE == SWAT_MODE_SIGMOID_) ? ((PRE && FwdTcCfg<D>::NSB == 3) ? 3 : 2) : 1;
     static constexpr int MMA_WARP = 0;
     static constexpr int TMA_WARP = 1;
     static constexpr int SCHED_WARP = 2;
     static constexpr int PV_WARP = 3;
     static constexpr int ACT_WARP0 = 4;
     static constexpr int PREP_WARP0 = ACT_WARP0 + 4 * ACT_WG;
-    static constexpr int THREADS = 32 * (PREP_WARP0 + 4);
+    static constexpr int THREADS = 32 * (PREP_WARP0 + (PRE ? 0 : 4));   // no prep warps when PRE
 };
 constexpr int FWD_PREP_BAR = 1;   // named barrier of the 128 prep threads
 
@@ -538,12 +542,12 @@ __device__ __forceinline__ float act_softmax_p(uint32_t s_addr, float sc2, float
 // PRE: Q and K arrive RoPE-rotated (copies in a workspace): the prep
 // warpgroup idles and the S MMAs wait for the TMA copies only.
 template <int D, int MODE, bool PRE>
-__global__ void __launch_bounds__(FwdRoles<MODE>::THREADS, 1)
+__global__ void __launch_bounds__(FwdRoles<D, MODE, PRE>::THREADS, 1)
 swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdArgs a)
 {
     using C = FwdTcCfg<D>;
-    using RL = FwdRoles<MODE>;
+    using RL = FwdRoles<D, MODE, PRE>;
     constexpr int NS = C::NSLOT;
     constexpr int FWD_PREP_WARP0 = RL::PREP_WARP0, FWD_MMA_WARP = RL::MMA_WARP, FWD_TMA_WARP = RL::TMA_WARP;
     constexpr int FWD_ACT_WARP0 = RL::ACT_WARP0;
@@ -832,7 +836,7 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         bool good = true;
         while (good && S.next_step(st)) {
             const int sb = st.step % NSB;
-            if (RL::ACT_WG == 2 && (st.step & 1) != aw) continue;   // the other warpgroup's tile
+            if (RL::ACT_WG > 1 && st.step % RL::ACT_WG != aw) continue;   // another warpgroup's tile
             const int i = st.i0 + r;
             const float slope = a.slopes ? __ldg(a.slopes + st.h) : 0.f;
             if (st.first) { m_used = -INFINITY; l_sum = 0.f; }
@@ -957,7 +961,8 @@ inline int launch_fwd_tc_t(const FwdArgs &a, void *ws, cudaStream_t stream)
     const long long items = (long long)a.B * a.H * ((a.N + 127) / 128);
     if (items >= (1LL << 31)) return -1;   // the schedule decodes item indices in 32 bits
     const int grid = (int)std::min<long long>(items, (long long)num_sms());
-    kern<<<grid, FwdRoles<MODE>::THREADS, C::SMEM, stream>>>(tq, tk, tv, a);
+    const int threads = pre ? FwdRoles<D, MODE, true>::THREADS : FwdRoles<D, MODE, false>::THREADS;
+    kern<<<grid, threads, C::SMEM, stream>>>(tq, tk, tv, a);
     return n + 1;
 }
 
