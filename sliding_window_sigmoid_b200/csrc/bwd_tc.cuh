@@ -56,6 +56,10 @@ struct BwdCfg {
     // -- S / dP MMAs, element-wise pass, gradient MMAs -- then spans three
     // half-steps), else two.
     static constexpr int NBUF = (3 * 128 + 2 * ACC_COLS <= 512 && ROLE != BWD_ROLE_DSUM) ? 3 : 2;
+    // activation warpgroups: one per buffer (half-step hs goes to warpgroup
+    // hs % NWG and buffer hs % NBUF, so a warpgroup always meets the same
+    // buffer and waits on its barriers in order)
+    static constexpr int NWG = NBUF;
     static constexpr int PD_COLS = (ROLE == BWD_ROLE_DKDV) ? 64 : (ROLE == BWD_ROLE_DQ ? 32 : 0);
     static constexpr bool SEP_PD = NBUF == 2 && PD_COLS > 0 && 256 + 2 * PD_COLS + 2 * ACC_COLS <= 512;
     static constexpr int ACC_BASE = NBUF * 128 + (SEP_PD ? 2 * PD_COLS : 0);
@@ -67,16 +71,17 @@ struct BwdCfg {
     static constexpr int OFF_ROT = OFF_B2 + NST * TILE;        // float2 [2][D/2] prep bases
     static constexpr int OFF_TH = OFF_ROT + 2 * (D / 2) * 8;   // double [D/2]
     static constexpr int OFF_THF = OFF_TH + (D / 2) * 8;       // float [D/2]
-    static constexpr int OFF_A0 = OFF_THF + (D / 2) * 4;       // float [2 wg][2][D/2] epilogue base angles
-    static constexpr int OFF_ROWS = OFF_A0 + 4 * (D / 2) * 4;  // float [2 wg][2 buf][128]: lse, D of 64 queries
-    static constexpr int OFF_DSUM = OFF_ROWS + 2 * 2 * 128 * 4; // float [2 item][2 wg][128]
-    static constexpr int OFF_BAR = OFF_DSUM + 2 * 2 * 128 * 4;
+    static constexpr int OFF_A0 = OFF_THF + (D / 2) * 4;       // float [3 wg][2][D/2] epilogue base angles
+    static constexpr int OFF_ROWS = OFF_A0 + 6 * (D / 2) * 4;  // float [3 wg][2 buf][128]: lse, D of 64 queries
+    static constexpr int OFF_DSUM = OFF_ROWS + 3 * 2 * 128 * 4; // float [2 item][3 wg][128]
+    static constexpr int OFF_BAR = OFF_DSUM + 2 * 3 * 128 * 4;
     static constexpr int NBAR = 3 * 2 + 4 * 4 + 3 * 3 + 4 * 2 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack for 1024-B alignment
     static_assert(OFF_BAR % 8 == 0, "barrier alignment");
     static_assert(SMEM <= 232448, "shared memory per CTA");
     static_assert(NST <= 4 && NBUF <= 3, "barrier arrays");
+    static_assert(ROLE != BWD_ROLE_DSUM || NWG == 2, "D_i partials: one half per warpgroup per step");
 };
 
 // Inverse RoPE of one accumulator row held in TMEM (fp32, D columns), for a
@@ -340,7 +345,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             sm100::mbar_init(stat_free + s, 1);
             sm100::mbar_init(acc_full + s, 1);
             sm100::mbar_init(acc_free + s, 128);
-            sm100::mbar_init(dsum_full + s, 256);
+            sm100::mbar_init(dsum_full + s, 128 * C::NWG);
             sm100::mbar_init(dsum_free + s, 128);
         }
         for (int s = 0; s < 3; ++s) {
@@ -521,9 +526,10 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             mbar_wait_drain(drain_g, 0);
         }
         __syncwarp();
-    } else if (warp >= BWD_ACT_WARP0 && warp < BWD_PREP_WARP0) {
+    } else if (warp >= BWD_ACT_WARP0 && warp < BWD_ACT_WARP0 + 4 * C::NWG) {
         // ------------------------------------------------------------ activation + epilogue
-        const int w = (warp - BWD_ACT_WARP0) / 4;                 // warpgroup = half of every step
+        constexpr int NWG = C::NWG;
+        const int w = (warp - BWD_ACT_WARP0) / 4;                 // warpgroup: half-steps hs = w mod NWG
         const int r = 32 * (warp % 4) + lane;                     // stationary row (= TMEM lane)
         const int wtid = threadIdx.x - 32 * (BWD_ACT_WARP0 + 4 * w);   // 0..127
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
@@ -534,12 +540,15 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
         struct PendE { int k, b, h, kvh, row0; };
         PendE pend{};
         bool has_pend = false;
+        int nep = 0, nmine = 0;                                   // epilogues / half-steps done here
         auto epilogue = [&](const PendE &p) -> bool {
             if (ROLE == BWD_ROLE_DSUM) {
                 const int ib = p.k & 1;
                 const bool ok = sm100::mbar_wait(dsum_full + ib, (p.k >> 1) & 1, abort_flag);
                 if (named_bar_or(2 + w, 128, !ok)) return false;
-                const float dsum = sDsum[(ib * 2 + 0) * 128 + r] + sDsum[(ib * 2 + 1) * 128 + r];
+                float dsum = 0.f;
+#pragma unroll
+                for (int j = 0; j < NWG; ++j) dsum += sDsum[(ib * NWG + j) * 128 + r];
                 const int i = p.row0 + r;
                 if (i < a.N) a.Dws[((size_t)p.b * a.H + p.h) * a.N + i] = dsum;
                 sm100::mbar_arrive(dsum_free + ib);
@@ -549,7 +558,8 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             const bool ok = sm100::mbar_wait(acc_full + ab, (p.k / NACC) & 1, abort_flag);
             if (named_bar_or(2 + w, 128, !ok)) return false;
             sm100::tc_fence_after();
-            float *A0 = sA0 + (w * 2 + ((p.k >> 1) & 1)) * (D / 2);
+            float *A0 = sA0 + (w * 2 + (nep & 1)) * (D / 2);        // the previous epilogue's set stays intact
+            ++nep;
             if (a.use_rope && wtid < D / 2) {
                 const double two_pi = 6.283185307179586476925286766559;
                 const double x = (double)p.row0 * sTh[wtid];
@@ -583,11 +593,13 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                 if (ROLE == BWD_ROLE_DQ) drow = a.Dws[((size_t)it.b * a.H + it.h) * a.N + row];
             }
             float dsum = 0.f;
+            // epilogue of this item: the warpgroup of its last half-step (2 groups: by item parity)
+            const int ep_w = (NWG == 2) ? (k & 1) : ((2 * (ts + it.T - 1) + 1) % NWG);
             // ALiBi slope of each step's query head, loaded one step ahead
             int head_n, pos_n;
             bwd_stream<ROLE>(it, G, 0, head_n, pos_n);
             float slope_n = a.slopes ? __ldg(a.slopes + (ROLE == BWD_ROLE_DKDV ? head_n : it.h)) : 0.f;
-            for (int t = 0; t < it.T; ++t, ++ts) {
+            for (int t = 0; good && t < it.T; ++t, ++ts) {
                 int head, pos0;
                 bwd_stream<ROLE>(it, G, t, head, pos0);
                 const float slope = slope_n;
@@ -595,11 +607,14 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                     bwd_stream<ROLE>(it, G, t + 1, head_n, pos_n);
                     slope_n = __ldg(a.slopes + head_n);
                 }
-                const int cb = pos0 + 64 * w;                         // first streamed row of this half
+                for (int h = 0; h < 2; ++h) {
+                const int hsm = 2 * ts + h;                           // this half-step
+                if (hsm % NWG != w) continue;
+                const int cb = pos0 + 64 * h;                         // first streamed row of this half
                 const float *colL = nullptr, *colD = nullptr;
                 if (!sig && ROLE == BWD_ROLE_DKDV) {
                     // lse (log2 units) and D of the 64 queries of this half
-                    float *rows = sRows + (w * 2 + (ts & 1)) * 128;
+                    float *rows = sRows + (w * 2 + (nmine & 1)) * 128;
                     const int c = wtid & 63, iq = cb + c;
                     float val = 0.f;
                     if (iq < a.N) {
@@ -633,7 +648,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                 }
                 // decisions to stop are taken by the whole warpgroup (it also meets at
                 // named barriers), so no warp waits at one that the others left
-                const int hsm = 2 * ts + w, bf = hsm % C::NBUF;        // this half-step and its buffer
+                const int bf = hsm % C::NBUF;                         // its TMEM buffer
                 const bool ok = sm100::mbar_wait(x_full + bf, (hsm / C::NBUF) & 1, abort_flag);
                 if (named_bar_or(2 + w, 128, !ok)) { good = false; break; }
                 sm100::tc_fence_after();
@@ -658,6 +673,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                 sm100::tmem_wait_st();
                 sm100::tc_fence_before();
                 sm100::mbar_arrive(p_full + bf);
+                ++nmine;
                 if (has_pend) {
                     has_pend = false;
                     if (!epilogue(pend)) { good = false; break; }
@@ -669,14 +685,15 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                             const bool okf = sm100::mbar_wait(dsum_free + ib, ((k >> 1) - 1) & 1, abort_flag);
                             if (named_bar_or(2 + w, 128, !okf)) { good = false; break; }
                         }
-                        sDsum[(ib * 2 + w) * 128 + r] = dsum;
+                        sDsum[(ib * NWG + w) * 128 + r] = dsum;
                         sm100::mbar_arrive(dsum_full + ib);
                     }
-                    if ((k & 1) == w) {
+                    if (w == ep_w) {
                         pend = PendE{k, it.b, it.h, it.kvh, it.row0};
                         has_pend = true;
                     }
                 }
+                }   // half
             }
         }
         if (good && has_pend) epilogue(pend);
