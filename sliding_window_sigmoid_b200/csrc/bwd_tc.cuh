@@ -15,20 +15,22 @@
 //         tiles of every query head of the group: S^T = K'Q'^T, dP^T = V dO^T,
 //         dV += P^T dO, dK' += dS^T Q'.
 //   DSUM  (softmax) the DQ products without dQ': D_i = sum_j p_ij dP_ij.
-// Each streamed tile is processed as two 64-column half-steps; half h of
-// every step goes to activation warpgroup h, which owns TMEM buffer h, so the
-// element-wise work of one half overlaps the MMAs of the other.
+// Each streamed tile is processed as two 64-column half-steps; half-step
+// hs goes to TMEM buffer hs % NBUF and activation warpgroup hs % NWG
+// (NWG = NBUF: 3 for dq at d 64, else 2), so the element-wise pass of one
+// half-step overlaps the MMAs of the next ones.
 // Warp roles (512 threads, one CTA per SM):
-//   warp 0     issues S / dP of each half-step (X MMAs) into TMEM buffer h.
+//   warp 0     issues S / dP of each half-step (X MMAs) into its TMEM buffer.
 //   warp 1     TMA: stationary tile pair per item, streamed pairs into a ring.
 //   warp 3     issues the gradient MMAs (dV, dK', dQ') of each half-step.
-//   warps 4-11 two activation warpgroups (one TMEM lane = one row per thread);
-//              the epilogue of item k runs in warpgroup k % 2, deferred until
-//              after its next half-step.
-//   warps 12-15 set-up only. Q and K arrive RoPE-rotated: a small kernel
+//   warps 4..  NWG activation warpgroups (one TMEM lane = one row per
+//              thread); the epilogue of an item runs in one of them,
+//              deferred until after its next half-step.
+//   others     set-up only. Q and K arrive RoPE-rotated: a small kernel
 //              writes rotated copies into the workspace first.
-// TMEM columns: [128 h, 128 h + 64) S half, [128 h + 64, 128 h + 128) dP half
-// (their first 32 columns then hold bf16 P and dS), accumulators from 256.
+// TMEM columns: buffer b = [128 b, 128 b + 128): S half, then dP half (bf16
+// P and dS over their first 32 columns, or in columns of their own);
+// accumulators after the buffers.
 #pragma once
 #include "fwd_tc.cuh"
 #include "rope_rows.cuh"
