@@ -73,8 +73,8 @@ struct BwdCfg {
     static constexpr int OFF_ROT = OFF_B2 + NST * TILE;        // float2 [2][D/2] prep bases
     static constexpr int OFF_TH = OFF_ROT + 2 * (D / 2) * 8;   // double [D/2]
     static constexpr int OFF_THF = OFF_TH + (D / 2) * 8;       // float [D/2]
-    static constexpr int OFF_A0 = OFF_THF + (D / 2) * 4;       // float [3 wg][2][D/2] epilogue base angles
-    static constexpr int OFF_ROWS = OFF_A0 + 6 * (D / 2) * 4;  // float [3 wg][2 buf][128]: lse, D of 64 queries
+    static constexpr int OFF_A0 = OFF_THF + (D / 2) * 4;       // float [3 wg][4 warps][D/2] epilogue base angles
+    static constexpr int OFF_ROWS = OFF_A0 + 12 * (D / 2) * 4; // float [3 wg][2 buf][128]: lse, D of 64 queries
     static constexpr int OFF_DSUM = OFF_ROWS + 3 * 2 * 128 * 4; // float [2 item][3 wg][128]
     static constexpr int OFF_BAR = OFF_DSUM + 2 * 3 * 128 * 4;
     static constexpr int NBAR = 3 * 2 + 4 * 4 + 3 * 3 + 4 * 2 + 2;
@@ -542,12 +542,18 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
         struct PendE { int k, b, h, kvh, row0; };
         PendE pend{};
         bool has_pend = false;
-        int nep = 0, nmine = 0;                                   // epilogues / half-steps done here
+        int nmine = 0;                                            // half-steps done here
+        // Stop decisions (abort) are taken per warp, except where the warpgroup
+        // meets at a named barrier after them (dk/dv softmax: per-column rows).
+        constexpr bool WG_BAR = (ROLE == BWD_ROLE_DKDV && MODE == SWAT_MODE_SOFTMAX_);
+        auto stop_any = [&](bool v) -> bool {
+            return WG_BAR ? named_bar_or(2 + w, 128, v) : (__any_sync(0xffffffffu, v) != 0);
+        };
         auto epilogue = [&](const PendE &p) -> bool {
             if (ROLE == BWD_ROLE_DSUM) {
                 const int ib = p.k & 1;
                 const bool ok = sm100::mbar_wait(dsum_full + ib, (p.k >> 1) & 1, abort_flag);
-                if (named_bar_or(2 + w, 128, !ok)) return false;
+                if (stop_any(!ok)) return false;
                 float dsum = 0.f;
 #pragma unroll
                 for (int j = 0; j < NWG; ++j) dsum += sDsum[(ib * NWG + j) * 128 + r];
@@ -558,16 +564,19 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             }
             const int ab = p.k % NACC;
             const bool ok = sm100::mbar_wait(acc_full + ab, (p.k / NACC) & 1, abort_flag);
-            if (named_bar_or(2 + w, 128, !ok)) return false;
+            if (stop_any(!ok)) return false;
             sm100::tc_fence_after();
-            float *A0 = sA0 + (w * 2 + (nep & 1)) * (D / 2);        // the previous epilogue's set stays intact
-            ++nep;
-            if (a.use_rope && wtid < D / 2) {
-                const double two_pi = 6.283185307179586476925286766559;
-                const double x = (double)p.row0 * sTh[wtid];
-                A0[wtid] = (float)(x - rint(x / two_pi) * two_pi);
+            // base angles of the item's rows, one copy per warp (no warpgroup barrier)
+            float *A0 = sA0 + (w * 4 + (warp % 4)) * (D / 2);
+            if (a.use_rope) {
+                __syncwarp();   // the previous epilogue's reads of this copy are done
+                for (int t = lane; t < D / 2; t += 32) {
+                    const double two_pi = 6.283185307179586476925286766559;
+                    const double x = (double)p.row0 * sTh[t];
+                    A0[t] = (float)(x - rint(x / two_pi) * two_pi);
+                }
+                __syncwarp();
             }
-            sm100::named_bar_sync(2 + w, 128);
             const uint32_t acc = tmem + lane_base + C::ACC_BASE + ab * C::ACC_COLS;
             const int row = p.row0 + r;
             if (ROLE == BWD_ROLE_DQ) {
@@ -648,16 +657,14 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                     b0 = slope * (float)rd * bmul;
                     bstep = -slope * bmul;
                 }
-                // decisions to stop are taken by the whole warpgroup (it also meets at
-                // named barriers), so no warp waits at one that the others left
                 const int bf = hsm % C::NBUF;                         // its TMEM buffer
                 const bool ok = sm100::mbar_wait(x_full + bf, (hsm / C::NBUF) & 1, abort_flag);
-                if (named_bar_or(2 + w, 128, !ok)) { good = false; break; }
+                if (stop_any(!ok)) { good = false; break; }
                 sm100::tc_fence_after();
                 if (C::SEP_PD && hsm >= C::NBUF) {
                     // P / dS columns of this buffer: read by the previous half-step's gradient MMAs
                     const bool okp = sm100::mbar_wait(buf_free + bf, ((hsm / C::NBUF) - 1) & 1, abort_flag);
-                    if (named_bar_or(2 + w, 128, !okp)) { good = false; break; }
+                    if (stop_any(!okp)) { good = false; break; }
                     sm100::tc_fence_after();
                 }
                 const uint32_t x_addr = tmem + lane_base + bf * 128;
@@ -685,7 +692,7 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                         const int ib = k & 1;
                         if (k >= 2) {
                             const bool okf = sm100::mbar_wait(dsum_free + ib, ((k >> 1) - 1) & 1, abort_flag);
-                            if (named_bar_or(2 + w, 128, !okf)) { good = false; break; }
+                            if (stop_any(!okf)) { good = false; break; }
                         }
                         sDsum[(ib * NWG + w) * 128 + r] = dsum;
                         sm100::mbar_arrive(dsum_full + ib);
