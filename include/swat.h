@@ -206,6 +206,15 @@ SWAT_API const char *swat_status_string(int status);
  * `stream`. Returns SWAT_ERR_CUDA if the read fails. */
 SWAT_API int swat_get_device_status(void *stream);
 
+/* Failure-path check (no counterpart in the pages): launches one kernel
+ * whose thread waits for an mbarrier phase that nothing completes, bounded
+ * by limit_ns of device time, exactly as the attention kernels bound their
+ * waits. It then records SWAT_ERR_TIMEOUT in the device status word and
+ * returns; the context stays usable. Read the result with
+ * swat_get_device_status(). limit_ns in [1e3, 2e9], else SWAT_ERR_INVALID_ARG
+ * before any launch. */
+SWAT_API int swat_check_wait_timeout(long long limit_ns, void *stream);
+
 /* Number of kernel launches the library has issued in this process (host
  * counter; lets a caller count device work done through this ABI). */
 SWAT_API long long swat_launch_count(void);

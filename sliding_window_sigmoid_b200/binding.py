@@ -28,7 +28,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20   # SWA_DECODE_NOALLOC_SCRATCH_BYTES
 
 EXPORTED = ["swat_attn_fwd", "swat_attn_fwd_workspace_bytes", "swat_attn_fwd_ws", "swat_attn_bwd_workspace_bytes", "swat_attn_bwd", "swa_cache_fill",
             "swa_decode_step", "swa_decode_workspace_bytes", "swa_decode_step_noalloc", "swat_status_string",
-            "swat_get_device_status", "swat_launch_count"]
+            "swat_get_device_status", "swat_launch_count", "swat_check_wait_timeout"]
 
 
 class SwatError(RuntimeError):
@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
     L.swat_status_string.restype = ctypes.c_char_p
     L.swat_get_device_status.argtypes = [P]
     L.swat_get_device_status.restype = I
+    L.swat_check_wait_timeout.argtypes = [LL, P]
+    L.swat_check_wait_timeout.restype = I
     L.swat_launch_count.argtypes = []
     L.swat_launch_count.restype = LL
     _lib = L
@@ -257,6 +259,11 @@ def status_string(code: int) -> str:
 
 def device_status(stream=None) -> int:
     return int(lib().swat_get_device_status(_stream(stream)))
+
+
+def check_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Runs the bounded-wait failure path once (see swat_check_wait_timeout)."""
+    _check("swat_check_wait_timeout", lib().swat_check_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def launch_count() -> int:

@@ -81,6 +81,34 @@ int swat_get_device_status(void *stream)
 }  // extern "C"
 
 namespace {
+// One thread waits, bounded by limit_ns of %globaltimer, for the first phase
+// of an mbarrier that nothing arrives on: the same bounded-wait path every
+// tensor-core kernel takes, ending in SWAT_ERR_TIMEOUT in the status word.
+__global__ void swat_wait_timeout_kernel(long long limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        swat::sm100::mbar_init(&bar, 1);
+        swat::sm100::fence_mbar_init();
+        const uint64_t t0 = swat::sm100::globaltimer();
+        while (!swat::sm100::mbar_try_wait(&bar, 0)) {
+            if (swat::sm100::globaltimer() - t0 > (uint64_t)limit_ns) {
+                swat::record_status(SWAT_ERR_TIMEOUT);
+                break;
+            }
+        }
+    }
+}
+}  // namespace
+
+extern "C" int swat_check_wait_timeout(long long limit_ns, void *stream)
+{
+    if (limit_ns < 1000 || limit_ns > 2000000000LL) return SWAT_ERR_INVALID_ARG;
+    swat_wait_timeout_kernel<<<1, 32, 0, S(stream)>>>(limit_ns);
+    return after_launch(1);
+}
+
+namespace {
 // The forward with an optional workspace for RoPE-rotated copies of Q and K.
 int attn_fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, void *workspace,
                   int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,

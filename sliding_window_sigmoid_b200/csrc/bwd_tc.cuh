@@ -54,10 +54,10 @@ struct BwdCfg {
     // only for the element-wise pass, not for the gradient MMAs), else over
     // the S / dP halves.
     // TMEM buffers of S / dP halves (128 columns each) in flight: three where
-    // they fit next to two accumulator sets (the dependency chain of a buffer
+    // they fit next to one accumulator set (the dependency chain of a buffer
     // -- S / dP MMAs, element-wise pass, gradient MMAs -- then spans three
     // half-steps), else two.
-    static constexpr int NBUF = (3 * 128 + 2 * ACC_COLS <= 512 && ROLE != BWD_ROLE_DSUM) ? 3 : 2;
+    static constexpr int NBUF = (ROLE != BWD_ROLE_DSUM && 3 * 128 + ACC_COLS <= 512) ? 3 : 2;
     // activation warpgroups: one per buffer (half-step hs goes to warpgroup
     // hs % NWG and buffer hs % NBUF, so a warpgroup always meets the same
     // buffer and waits on its barriers in order)

@@ -116,3 +116,10 @@ def test_bwd_and_decode_reject_invalid_arguments(L):
     st = L.swa_cache_fill(FAKE, FAKE, FAKE, FAKE, None, None, 1, 2, 8, 64, 0, 0, 0, 1e4, 0, None)
     assert st == -1                                                      # window 0
     assert binding.launch_count() == before
+
+
+def test_check_wait_timeout_rejects_bad_limits_before_launch(L):
+    n0 = binding.launch_count()
+    for bad in (0, 999, 2_000_000_001, -5):
+        assert L.swat_check_wait_timeout(bad, None) == -1
+    assert binding.launch_count() == n0
