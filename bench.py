@@ -330,42 +330,64 @@ def run_swat(args):
 
 def bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, fws, kw):
     """Same step through the public API with host buffers: every step copies
-    Q, K, V, dO from pinned host memory and reads O, dQ, dK, dV back."""
+    Q, K, V, dO from pinned host memory and reads O, dQ, dK, dV back. Steps
+    are pipelined over three streams (host-to-device copies, compute,
+    device-to-host copies) with two device buffer sets, so the copies of
+    neighbouring steps overlap each other and the compute, as a training
+    loop that streams batches would run them."""
     import torch
     from sliding_window_sigmoid_b200 import binding
+    dev = q.device
     hq, hk, hv, hdo = [t.cpu().pin_memory() for t in (q, k, v, do)]
     ho, hdq, hdk, hdv = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, dq, dk, dv)]
-    dq_in, dk_in, dv_in, ddo_in = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
-                                   torch.empty_like(do))
+    ins = [tuple(torch.empty_like(t) for t in (q, k, v, do)) for _ in range(2)]
+    outs = [(o, dq, dk, dv), tuple(torch.empty_like(t) for t in (o, dq, dk, dv))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_ready, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def e2e_step():
-        dq_in.copy_(hq, non_blocking=True)
-        dk_in.copy_(hk, non_blocking=True)
-        dv_in.copy_(hv, non_blocking=True)
-        ddo_in.copy_(hdo, non_blocking=True)
-        binding.attn_fwd(dq_in, dk_in, dv_in, out=o, workspace=fws, **kw)
-        binding.attn_bwd(dq_in, dk_in, dv_in, o, None, ddo_in, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
-        ho.copy_(o, non_blocking=True)
-        hdq.copy_(dq, non_blocking=True)
-        hdk.copy_(dk, non_blocking=True)
-        hdv.copy_(dv, non_blocking=True)
+    def run(n_steps):
+        for t in range(n_steps):
+            j = t % 2
+            if t >= 2:
+                s_in.wait_event(comp_done[j])          # inputs set j free again
+            with torch.cuda.stream(s_in):
+                for dst, src in zip(ins[j], (hq, hk, hv, hdo)):
+                    dst.copy_(src, non_blocking=True)
+                in_ready[j].record(s_in)
+            stream.wait_event(in_ready[j])
+            if t >= 2:
+                stream.wait_event(out_done[j])         # outputs set j read back
+            iq, ik, iv, ido = ins[j]
+            oo, odq, odk, odv = outs[j]
+            binding.attn_fwd(iq, ik, iv, out=oo, workspace=fws, stream=stream, **kw)
+            binding.attn_bwd(iq, ik, iv, oo, None, ido, dq=odq, dk=odk, dv=odv, workspace=ws, stream=stream,
+                             **kw)
+            comp_done[j].record(stream)
+            s_out.wait_event(comp_done[j])
+            with torch.cuda.stream(s_out):
+                for dst, src in zip((ho, hdq, hdk, hdv), outs[j]):
+                    dst.copy_(src, non_blocking=True)
+                out_done[j].record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    run(max(1, args.warmup))
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    run(args.steps)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     nbytes = lambda ts: sum(t.numel() * t.element_size() for t in ts)
     e2e = {"value": job_value(step_flops, world, args.steps, e2e_ms), "unit": "TFLOP/s",
            "h2d_bytes_per_step": nbytes((hq, hk, hv, hdo)),
-           "d2h_bytes_per_step": nbytes((ho, hdq, hdk, hdv))}
+           "d2h_bytes_per_step": nbytes((ho, hdq, hdk, hdv)),
+           "pipelined": "h2d / compute / d2h streams, 2 buffer sets"}
     return e2e
 
 
