@@ -258,7 +258,7 @@ def run_swat(args):
 
     def step():
         binding.attn_fwd(q, k, v, out=o, workspace=fws, **kw)
-        binding.attn_bwd(q, k, v, o, None, do, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+        binding.attn_bwd(q, k, v, o, None, do, dq=dq, dk=dk, dv=dv, workspace=ws, qk_rot=fws, **kw)
 
     for _ in range(args.warmup):
         step()
@@ -281,7 +281,7 @@ def run_swat(args):
         evs[i][0].record(stream)
         binding.attn_fwd(q, k, v, out=o, workspace=fws, **kw)
         evs[i][1].record(stream)
-        binding.attn_bwd(q, k, v, o, None, do, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+        binding.attn_bwd(q, k, v, o, None, do, dq=dq, dk=dk, dv=dv, workspace=ws, qk_rot=fws, **kw)
         evs[i][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
@@ -361,8 +361,8 @@ def bench_e2e(args, world, stream, step_flops, q, k, v, do, o, dq, dk, dv, ws, f
             iq, ik, iv, ido = ins[j]
             oo, odq, odk, odv = outs[j]
             binding.attn_fwd(iq, ik, iv, out=oo, workspace=fws, stream=stream, **kw)
-            binding.attn_bwd(iq, ik, iv, oo, None, ido, dq=odq, dk=odk, dv=odv, workspace=ws, stream=stream,
-                             **kw)
+            binding.attn_bwd(iq, ik, iv, oo, None, ido, dq=odq, dk=odk, dv=odv, workspace=ws, qk_rot=fws,
+                             stream=stream, **kw)
             comp_done[j].record(stream)
             s_out.wait_event(comp_done[j])
             with torch.cuda.stream(s_out):

@@ -122,6 +122,18 @@ SWAT_API int swat_attn_bwd(const void *q, const void *k, const void *v, const vo
                   int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
                   const float *slopes, float rope_base, int dtype, void *stream);
 
+/* swat_attn_bwd reusing the forward's rotated copies: qk_rot is the
+ * workspace of a swat_attn_fwd_ws call on the same q and k with the same
+ * B, H, Hkv, N, d and rope_base (bf16), and must still hold what that call
+ * wrote; the backward then skips its own RoPE pass (a training step rotates
+ * Q and K once). Same operation, arguments and results as swat_attn_bwd
+ * otherwise; `workspace` is still required. SWAT_ERR_INVALID_ARG for a
+ * missing or misaligned qk_rot (bf16 with RoPE on). */
+SWAT_API int swat_attn_bwd_rotated(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dout, void *dq, void *dk, void *dv, void *workspace, const void *qk_rot,
+                  int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
+                  const float *slopes, float rope_base, int dtype, void *stream);
+
 /* Ring-buffer KV cache ([SWA] ring-buffer paragraph, [SWA] "Attention sink"):
  *   k_cache, v_cache [B, Hkv, window, d]: slot s holds the token whose
  *           position p satisfies p mod window == s (the newest such p); keys

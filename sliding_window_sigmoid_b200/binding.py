@@ -26,7 +26,8 @@ _STATUS = {0: "SWAT_OK", -1: "SWAT_ERR_INVALID_ARG", -2: "SWAT_ERR_UNSUPPORTED",
 SCRATCH_LIMIT = -5
 NOALLOC_SCRATCH_BYTES = 16 << 20   # SWA_DECODE_NOALLOC_SCRATCH_BYTES
 
-EXPORTED = ["swat_attn_fwd", "swat_attn_fwd_workspace_bytes", "swat_attn_fwd_ws", "swat_attn_bwd_workspace_bytes", "swat_attn_bwd", "swa_cache_fill",
+EXPORTED = ["swat_attn_fwd", "swat_attn_fwd_workspace_bytes", "swat_attn_fwd_ws", "swat_attn_bwd_workspace_bytes", "swat_attn_bwd", "swat_attn_bwd_rotated",
+            "swa_cache_fill",
             "swa_decode_step", "swa_decode_workspace_bytes", "swa_decode_step_noalloc", "swat_status_string",
             "swat_get_device_status", "swat_launch_count", "swat_check_wait_timeout"]
 
@@ -60,6 +61,8 @@ def lib() -> ctypes.CDLL:
     L.swat_attn_bwd_workspace_bytes.restype = SZ
     L.swat_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, F, I, P]
     L.swat_attn_bwd.restype = I
+    L.swat_attn_bwd_rotated.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, F, I, P]
+    L.swat_attn_bwd_rotated.restype = I
     L.swa_cache_fill.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, LL, F, I, P]
     L.swa_cache_fill.restype = I
     L.swa_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, F, I, P]
@@ -168,8 +171,11 @@ def bwd_workspace_bytes(B, H, Hkv, N, d, dtype=BF16) -> int:
 
 def attn_bwd(q, k, v, o, lse, dout, *, window: int, n_sink: int = 0, mode: int = MODE_SIGMOID,
              slopes=None, rope_base: float = 10000.0, dq=None, dk=None, dv=None, workspace=None,
-             stream=None):
-    """Backward of attn_fwd. Returns (dq, dk, dv)."""
+             qk_rot=None, stream=None):
+    """Backward of attn_fwd. Returns (dq, dk, dv).
+
+    qk_rot: the workspace given to attn_fwd for the same q and k (its rotated
+    copies are reused: swat_attn_bwd_rotated), or None (swat_attn_bwd)."""
     B, N, H, d = q.shape
     Hkv = k.shape[2]
     dev = q.device
@@ -181,9 +187,15 @@ def attn_bwd(q, k, v, o, lse, dout, *, window: int, n_sink: int = 0, mode: int =
         nbytes = bwd_workspace_bytes(B, H, Hkv, N, d, _dtype_code(q))
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
     sl = _slopes(slopes, H, dev)
+    rest = (B, H, Hkv, N, d, window, n_sink, mode, _ptr(sl), float(rope_base), _dtype_code(q),
+            _stream(stream))
+    if qk_rot is not None:
+        st = lib().swat_attn_bwd_rotated(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _ptr(qk_rot), *rest)
+        _check("swat_attn_bwd_rotated", st)
+        return dq, dk, dv
     st = lib().swat_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
-                             _ptr(dk), _ptr(dv), _ptr(workspace), B, H, Hkv, N, d, window, n_sink,
-                             mode, _ptr(sl), float(rope_base), _dtype_code(q), _stream(stream))
+                             _ptr(dk), _ptr(dv), _ptr(workspace), *rest)
     _check("swat_attn_bwd", st)
     return dq, dk, dv
 

@@ -182,8 +182,11 @@ size_t swat_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int d, int dt
     return D + extra;
 }
 
-int swat_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
-                  const void *dout, void *dq, void *dk, void *dv, void *workspace,
+}  // extern "C"
+
+namespace {
+int attn_bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dout, void *dq, void *dk, void *dv, void *workspace, const void *qk_rot,
                   int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
                   const float *slopes, float rope_base, int dtype, void *stream)
 {
@@ -211,7 +214,7 @@ int swat_attn_bwd(const void *q, const void *k, const void *v, const void *o, co
     }
     if (dtype == SWAT_BF16) {
         size_t D = ((size_t)B * H * N * sizeof(float) + 255) & ~(size_t)255;
-        int m = swat::launch_bwd_tc(a, (char *)workspace + D, S(stream));
+        int m = swat::launch_bwd_tc(a, (char *)workspace + D, qk_rot, S(stream));
         if (m < 0) return SWAT_ERR_CUDA;
         return after_launch(n + m);
     }
@@ -223,6 +226,28 @@ int swat_attn_bwd(const void *q, const void *k, const void *v, const void *o, co
     swat::swat_bwd_dq_simt_kernel<float><<<gq, swat::SIMT_THREADS, smem_q, S(stream)>>>(a);
     swat::swat_bwd_dkdv_simt_kernel<float><<<gk, swat::SIMT_THREADS, smem_k, S(stream)>>>(a);
     return after_launch(n + 2);
+}
+}  // namespace
+
+extern "C" {
+
+int swat_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                  int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
+                  const float *slopes, float rope_base, int dtype, void *stream)
+{
+    return attn_bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, nullptr, B, H, Hkv, N, d, window, n_sink,
+                         mode, slopes, rope_base, dtype, stream);
+}
+
+int swat_attn_bwd_rotated(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                          const void *dout, void *dq, void *dk, void *dv, void *workspace, const void *qk_rot,
+                          int B, int H, int Hkv, int N, int d, int window, int n_sink, int mode,
+                          const float *slopes, float rope_base, int dtype, void *stream)
+{
+    if (dtype == SWAT_BF16 && rope_base > 0.f && (!qk_rot || !aligned16(qk_rot))) return SWAT_ERR_INVALID_ARG;
+    return attn_bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, dtype == SWAT_BF16 ? qk_rot : nullptr,
+                         B, H, Hkv, N, d, window, n_sink, mode, slopes, rope_base, dtype, stream);
 }
 
 int swa_cache_fill(const void *k, const void *v, void *k_cache, void *v_cache,

@@ -737,12 +737,16 @@ inline bool launch_bwd_role(const BwdArgs &a, const CUtensorMap &tq, const CUten
 }
 
 template <int D, int MODE>
-inline int launch_bwd_tc_t(const BwdArgs &a, void *extra_ws, cudaStream_t stream)
+inline int launch_bwd_tc_t(const BwdArgs &a, void *extra_ws, const void *qk_rot, cudaStream_t stream)
 {
     int n = 0;
     const void *qr = a.q, *kr = a.k;
-    if (a.use_rope)   // rotated copies of Q and K in the workspace
+    if (a.use_rope && qk_rot) {   // the forward's rotated copies (same layout)
+        qr = qk_rot;
+        kr = reinterpret_cast<const char *>(qk_rot) + align256((size_t)a.B * a.N * a.H * D * 2);
+    } else if (a.use_rope) {      // rotated copies of Q and K in the workspace
         n += launch_rope_copies<D>(a.q, a.k, extra_ws, a.B, a.H, a.Hkv, a.N, a.log2_base, stream, &qr, &kr);
+    }
     CUtensorMap tq, tk, tv, tdo;
     if (!make_tmap_bshd(&tq, qr, a.B, a.N, a.H, D) || !make_tmap_bshd(&tk, kr, a.B, a.N, a.Hkv, D) ||
         !make_tmap_bshd(&tv, a.v, a.B, a.N, a.Hkv, D) || !make_tmap_bshd(&tdo, a.dout, a.B, a.N, a.H, D))
@@ -763,14 +767,16 @@ inline size_t tc_bwd_extra_workspace(int B, int H, int Hkv, int N, int d)
 }
 
 // Returns the number of kernels launched, or -1 on a launch-configuration error.
-inline int launch_bwd_tc(const BwdArgs &a, void *extra_ws, cudaStream_t stream)
+// qk_rot: NULL, or the rotated copies a swat_attn_fwd_ws call wrote for
+// the same q and k (skips the rotation kernels).
+inline int launch_bwd_tc(const BwdArgs &a, void *extra_ws, const void *qk_rot, cudaStream_t stream)
 {
     if (a.d == 64)
-        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<64, SWAT_MODE_SIGMOID_>(a, extra_ws, stream)
-                                            : launch_bwd_tc_t<64, SWAT_MODE_SOFTMAX_>(a, extra_ws, stream);
+        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<64, SWAT_MODE_SIGMOID_>(a, extra_ws, qk_rot, stream)
+                                            : launch_bwd_tc_t<64, SWAT_MODE_SOFTMAX_>(a, extra_ws, qk_rot, stream);
     if (a.d == 128)
-        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<128, SWAT_MODE_SIGMOID_>(a, extra_ws, stream)
-                                            : launch_bwd_tc_t<128, SWAT_MODE_SOFTMAX_>(a, extra_ws, stream);
+        return a.mode == SWAT_MODE_SIGMOID_ ? launch_bwd_tc_t<128, SWAT_MODE_SIGMOID_>(a, extra_ws, qk_rot, stream)
+                                            : launch_bwd_tc_t<128, SWAT_MODE_SOFTMAX_>(a, extra_ws, qk_rot, stream);
     return -1;
 }
 

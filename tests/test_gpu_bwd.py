@@ -88,3 +88,23 @@ def test_full_size_swat_340m_bwd_sampled_rows():
     assert_bf16_close(np.stack([dv_np[b, j, h] for b, h, j in krows]), rv, "dv rows")
     for g in (dq_np, dk_np, dv_np):
         assert np.isfinite(g).all()
+
+
+@pytest.mark.parametrize("mode,H,Hkv,d", [(0, 4, 4, 64), (1, 8, 2, 128)])
+def test_bwd_reusing_forward_rotated_copies_is_identical(mode, H, Hkv, d):
+    """swat_attn_bwd_rotated with the forward workspace gives bit-identical
+    gradients to swat_attn_bwd (same rotation, same kernels)."""
+    B, N, w, s = 2, 333, 96, (4 if mode == 1 else 0)
+    scale = 1.0 / np.sqrt(d) if mode == 0 else 1.0
+    q, k, v, do = [t.to(DEV) for t in inputs.qkv(B, N, H, Hkv, d, seed=9, scale=scale, dtype=torch.bfloat16,
+                                                  with_dout=True)]
+    sl = inputs.balanced_alibi_slopes(H).to(DEV) if mode == 0 else None
+    kw = dict(window=w, n_sink=s, mode=mode, slopes=sl, rope_base=1e4)
+    fws = torch.empty(binding.fwd_workspace_bytes(B, H, Hkv, N, d), dtype=torch.uint8, device=DEV)
+    o, lse = binding.attn_fwd(q, k, v, workspace=fws, **kw)
+    g_ref = binding.attn_bwd(q, k, v, o, lse, do, **kw)
+    g_rot = binding.attn_bwd(q, k, v, o, lse, do, qk_rot=fws, **kw)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    for a, b in zip(g_ref, g_rot):
+        assert torch.equal(a, b)
