@@ -89,9 +89,12 @@ struct BwdCfg {
 // Inverse RoPE of one accumulator row held in TMEM (fp32, D columns), for a
 // row at absolute position pos0 + r; the angle is A0[t] + r theta_t (A0 is the
 // position pos0 reduced in fp64), reduced again in fp32 before __sincosf.
+// release: when non-null, arrived on (once per thread) as soon as the last
+// TMEM load has landed, so the accumulator can be reused during the stores.
 template <int D>
 __device__ __forceinline__ void unrotate_store_row(uint32_t taddr, int r, const float *A0, const float *THF,
-                                                   bool use_rope, __nv_bfloat16 *dst, bool store, float mul = 1.f)
+                                                   bool use_rope, __nv_bfloat16 *dst, bool store, float mul = 1.f,
+                                                   uint64_t *release = nullptr)
 {
     const float two_pi = 6.2831853071795865f, inv_two_pi = 0.15915494309189534f;
 #pragma unroll
@@ -99,6 +102,10 @@ __device__ __forceinline__ void unrotate_store_row(uint32_t taddr, int r, const 
         uint32_t v[32];
         sm100::tmem_ld32(taddr + 32 * k, v);
         sm100::tmem_wait_ld_dep(v);
+        if (release && k == D / 32 - 1) {
+            sm100::tc_fence_before();
+            sm100::mbar_arrive(release);
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -585,8 +592,10 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
             } else {
                 const size_t o = (((size_t)p.b * a.N + row) * a.Hkv + p.kvh) * D;
                 store_row_bf16_plain<D>(acc, reinterpret_cast<__nv_bfloat16 *>(a.dv) + o, row < a.N);
+                // dK' is read last: the accumulators are released after its final TMEM load
                 unrotate_store_row<D>(acc + D, r, A0, sThf, a.use_rope, reinterpret_cast<__nv_bfloat16 *>(a.dk) + o,
-                                      row < a.N, a.scale);
+                                      row < a.N, a.scale, acc_free + ab);
+                return true;
             }
             sm100::tc_fence_before();
             sm100::mbar_arrive(acc_free + ab);
@@ -700,6 +709,10 @@ swat_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_const
                     if (w == ep_w) {
                         pend = PendE{k, it.b, it.h, it.kvh, it.row0};
                         has_pend = true;
+                        if (NACC == 1) {   // one accumulator set: the next item's MMAs wait for it, so now
+                            has_pend = false;
+                            if (!epilogue(pend)) { good = false; break; }
+                        }
                     }
                 }
                 }   // half
