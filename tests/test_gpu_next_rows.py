@@ -42,7 +42,9 @@ def test_decode_after_prefill_equals_prefill_last_row(mode, H, Hkv, d, w, s, bas
     od = cache.step(q[:, N - 1].contiguous(), k[:, N - 1].contiguous(), v[:, N - 1].contiguous(), pos)
     torch.cuda.synchronize()
     assert binding.device_status() == 0
-    assert_bf16_close(od, o[:, N - 1], "decode vs prefill last row")
+    # both sides are rounded to bf16: allow the second rounding (half an ulp of |o|)
+    ref = o[:, N - 1].float().cpu().numpy()
+    assert_bf16_close(od, ref, "decode vs prefill last row", allowance=2.0 ** -8 * np.abs(ref))
 
 
 def test_forward_only_slopes_match_oracle():
