@@ -21,9 +21,22 @@ namespace swat {
 
 // Ring slots per CTA of the decode attention: long enough that the per-CTA
 // set-up (query rotation, final reduction) is small next to the streaming;
-// measured on B200 (batch 64, w 4096): 512 -> 67 %, 1024 -> 74 %, 2048 -> 76 %
-// of the copy bandwidth.
-constexpr int DEC_SLOTS_PER_SPLIT = 2048;
+// measured on B200 (batch 64, w 4096, sigmoid, no L2 prefetch): 512 -> 67 %,
+// 1024 -> 74 %, 2048 -> 76 % of the copy bandwidth; with the L2 prefetch
+// below, 1024 -> 85 % and 2048 -> 88 %.
+#ifndef SWAT_DEC_SLOTS
+#define SWAT_DEC_SLOTS 2048
+#endif
+constexpr int DEC_SLOTS_PER_SPLIT = SWAT_DEC_SLOTS;
+// Iterations of K/V rows the streaming kernel keeps on their way into L2
+// ahead of its own loads (bulk L2 prefetches of contiguous slot ranges).
+// Measured on B200 (batch 64, w 4096, 2048 slots per CTA): 0 -> 76 % / 72 %,
+// 1 to 3 -> 88 % / 79 %, 4 -> 85 % / 78 %, 8 -> 61 % / 58 % of the copy
+// bandwidth (sigmoid / softmax with sinks).
+#ifndef SWAT_DEC_PFD
+#define SWAT_DEC_PFD 2
+#endif
+constexpr int DEC_PREFETCH_ITERS = SWAT_DEC_PFD;
 constexpr int DEC_THREADS = 256;
 constexpr int DEC_MAX_G = 8;
 

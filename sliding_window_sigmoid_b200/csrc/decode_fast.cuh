@@ -75,6 +75,22 @@ swa_decode_attn_bf16_kernel(DecArgs a)
         __syncthreads();
     }
 
+    // ---- L2 prefetch: one thread keeps the CTA's next PFD iterations of K and
+    // V rows (contiguous slot ranges) on their way into L2 with bulk
+    // prefetches, so the warps' own loads mostly hit L2 and fewer bytes need
+    // to be in flight per warp; the first PFD go out before the query rotation.
+    constexpr int CROWS = U * NW * RPW;                // slots the CTA consumes per iteration
+    constexpr int PFD = DEC_PREFETCH_ITERS;            // iterations prefetched ahead
+    auto prefetch_rows = [&](int r0) {
+        if (r0 < s1) {
+            const uint32_t bytes = (uint32_t)(min(CROWS, s1 - r0) * D * 2);
+            sm100::bulk_prefetch_l2(kc + (size_t)r0 * D, bytes);
+            sm100::bulk_prefetch_l2(vc + (size_t)r0 * D, bytes);
+        }
+    };
+    if (PFD > 0 && threadIdx.x == 0)
+        for (int i = 0; i < PFD; ++i) prefetch_rows(s0 + i * CROWS);
+
     // ---- rotated queries of the group, this lane's 8 dimensions
     float q[G][8];
     {
@@ -117,7 +133,8 @@ swa_decode_attn_bf16_kernel(DecArgs a)
     const float my_slope = a.slopes ? __ldg(a.slopes + kvh * G + hh) : 0.f;
     float mh = -INFINITY, lh = 0.f;                   // softmax state of head hh (this lane's copy)
 
-    auto consume = [&](const uint4 &kr, const uint4 &vr, int delta, bool valid) {
+    // Score of one cache row for head hh (this lane's head after the exchange).
+    auto score = [&](const uint4 &kr, int delta) -> float {
         const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
         sm100::f2 kf[4];
 #pragma unroll
@@ -148,32 +165,14 @@ swa_decode_attn_bf16_kernel(DecArgs a)
         float x = s[0];
 #pragma unroll
         for (int off = HSPAN / 2; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-        x += my_slope * (float)delta;                 // score of head hh
-        float pw, f = 1.f;
-        if (MODE == SWAT_MODE_SIGMOID_) {
-            pw = valid ? fmaf(0.5f, sm100::tanh_approx(0.5f * x), 0.5f) : 0.f;
-        } else {
-            // lazy rescaling: keep the running maximum until a score exceeds it by 8
-            if (valid && x > mh + 8.f) {
-                f = (mh == -INFINITY) ? 0.f : __expf(mh - x);
-                mh = x;
-                lh *= f;
-            }
-            pw = valid ? __expf(x - mh) : 0.f;
-            lh += pw;
-        }
+        return x + my_slope * (float)delta;
+    };
+    // acc[g] += p_g v for one cache row, p_g taken from a lane of head g.
+    auto accumulate = [&](const uint4 &vr, float pw) {
         const uint32_t vw[4] = {vr.x, vr.y, vr.z, vr.w};
         sm100::f2 vf[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) vf[p] = {sm100::bf16lo(vw[p]), sm100::bf16hi(vw[p])};
-        if (MODE == SWAT_MODE_SOFTMAX_ && __any_sync(0xffffffffu, f != 1.f)) {
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float fg = __shfl_sync(0xffffffffu, f, grp * LPR + g * HSPAN);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[g][e] *= fg;
-            }
-        }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             const float pg = __shfl_sync(0xffffffffu, pw, grp * LPR + g * HSPAN);
@@ -186,6 +185,37 @@ swa_decode_attn_bf16_kernel(DecArgs a)
             }
         }
     };
+    // Rescales the accumulators of the heads whose running maximum moved.
+    auto rescale = [&](float f) {
+        if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float fg = __shfl_sync(0xffffffffu, f, grp * LPR + g * HSPAN);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[g][e] *= fg;
+            }
+        }
+    };
+    // One row: score, weight, accumulate. In softmax mode the running maximum
+    // is raised lazily (only when a score exceeds it by 8).
+    auto consume = [&](const uint4 &kr, const uint4 &vr, int delta, bool valid) {
+        const float x = score(kr, delta);
+        float pw;
+        if (MODE == SWAT_MODE_SIGMOID_) {
+            pw = valid ? fmaf(0.5f, sm100::tanh_approx(0.5f * x), 0.5f) : 0.f;
+        } else {
+            float f = 1.f;
+            if (valid && x > mh + 8.f) {
+                f = (mh == -INFINITY) ? 0.f : __expf(mh - x);
+                mh = x;
+                lh *= f;
+            }
+            pw = valid ? __expf(x - mh) : 0.f;
+            lh += pw;
+            rescale(f);
+        }
+        accumulate(vr, pw);
+    };
 
     // ---- ring slots of this split. Loop bounds are warp-uniform (the row
     // groups of a warp must take the same trip count: consume() shuffles
@@ -193,6 +223,7 @@ swa_decode_attn_bf16_kernel(DecArgs a)
     // is masked.
     constexpr int STRIDE = NW * RPW;
     for (int base = s0 + warp * RPW; base < s1; base += U * STRIDE) {
+        if (PFD > 0 && threadIdx.x == 0) prefetch_rows(base + PFD * CROWS);
         uint4 kr[U], vr[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -201,12 +232,41 @@ swa_decode_attn_bf16_kernel(DecArgs a)
             kr[u] = __ldg(reinterpret_cast<const uint4 *>(kc + (size_t)sl * D + 8 * li));
             vr[u] = __ldg(reinterpret_cast<const uint4 *>(vc + (size_t)sl * D + 8 * li));
         }
+        if constexpr (MODE == SWAT_MODE_SIGMOID_) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int slot = base + u * STRIDE + grp;
-            const int delta = (slot <= pm) ? pm - slot : pm - slot + w;   // distance of the position held
-            const bool valid = slot < s1 && (long long)delta <= P;
-            consume(kr[u], vr[u], delta, valid);
+            for (int u = 0; u < U; ++u) {
+                const int slot = base + u * STRIDE + grp;
+                const int delta = (slot <= pm) ? pm - slot : pm - slot + w;   // distance of the position held
+                const bool valid = slot < s1 && (long long)delta <= P;
+                consume(kr[u], vr[u], delta, valid);
+            }
+        } else {
+            // softmax: the U rows are scored first and the running maximum is
+            // raised at most once for the group (by its largest valid score),
+            // so the rows do not wait on one another through a branch
+            float x[U], xm = -INFINITY;
+            bool valid[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int slot = base + u * STRIDE + grp;
+                const int delta = (slot <= pm) ? pm - slot : pm - slot + w;
+                valid[u] = slot < s1 && (long long)delta <= P;
+                x[u] = score(kr[u], delta);
+                xm = valid[u] ? fmaxf(xm, x[u]) : xm;
+            }
+            float f = 1.f;
+            if (xm > mh + 8.f) {
+                f = (mh == -INFINITY) ? 0.f : __expf(mh - xm);
+                mh = xm;
+                lh *= f;
+            }
+            rescale(f);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float pw = valid[u] ? __expf(x[u] - mh) : 0.f;
+                lh += pw;
+                accumulate(vr[u], pw);
+            }
         }
     }
     // ---- sinks before the window (split 0)
