@@ -416,8 +416,10 @@ __device__ __forceinline__ uint32_t col_bits32(const RowMask &m, int c0)
 }
 
 // Sigmoid weights of 16 S columns into 8 packed bf16 pairs:
-// sigma(x) = 0.5 + 0.5 tanh(x / 2), x = s/sqrt(d) + slope (i - j); columns
-// whose bit in `m` is clear get P = 0.
+// sigma(x) = 0.5 + 0.5 tanh(x / 2), x = s/sqrt(d) + slope (i - j); with
+// MASKED, columns whose bit in `m` is clear get P = 0 (without, every column
+// of the chunk is in the key set).
+template <bool MASKED = true>
 __device__ __forceinline__ void sigmoid_chunk(const uint32_t (&v)[16], uint32_t (&pk)[8], sm100::f2 bias,
                                               sm100::f2 step2, sm100::f2 hs2, uint32_t m)
 {
@@ -429,8 +431,10 @@ __device__ __forceinline__ void sigmoid_chunk(const uint32_t (&v)[16], uint32_t 
         bias = sm100::add2(bias, step2);
         const sm100::f2 th = {sm100::tanh_approx(x.x), sm100::tanh_approx(x.y)};
         sm100::f2 p = sm100::fma2(th, half2, half2);
-        p.x = (m & (1u << (2 * e))) ? p.x : 0.f;
-        p.y = (m & (1u << (2 * e + 1))) ? p.y : 0.f;
+        if (MASKED) {
+            p.x = (m & (1u << (2 * e))) ? p.x : 0.f;
+            p.y = (m & (1u << (2 * e + 1))) ? p.y : 0.f;
+        }
         pk[e] = sm100::pack_bf16x2(p.x, p.y);
     }
 }
@@ -479,6 +483,31 @@ __device__ __forceinline__ void act_sigmoid_tile(uint32_t s_addr, float hs, floa
         sm100::tmem_wait_ld_dep16(v1);
         if (c0 + 32 < 128) sm100::tmem_ld16(s_addr + c0 + 32, v0);
         sigmoid_chunk_any(v1, s_addr, c0 + 16, step2, hs2, nh2, hb2, mk, rd_w0, window, sink_cols);
+        if (c0 + 32 < 128) sm100::tmem_wait_ld_dep16(v0);
+    }
+}
+
+// act_sigmoid_tile for a tile whose 128 x 128 (query, key) pairs are all in
+// the key set (interior band tiles): no masks, no chunk tests.
+__device__ __forceinline__ void act_sigmoid_tile_full(uint32_t s_addr, float hs, float hsl, int rd)
+{
+    const sm100::f2 hs2 = {hs, hs}, step2 = {-2.f * hsl, -2.f * hsl}, nh2 = {-hsl, -hsl};
+    const float hb0 = hsl * (float)rd;
+    const sm100::f2 hb2 = {hb0, hb0};
+    uint32_t v0[16], v1[16], pk[8];
+    sm100::tmem_ld16(s_addr, v0);
+    sm100::tmem_wait_ld_dep16(v0);
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+        sm100::tmem_ld16(s_addr + c0 + 16, v1);
+        const sm100::f2 cp0 = {(float)c0, (float)(c0 + 1)};
+        sigmoid_chunk<false>(v0, pk, sm100::fma2(cp0, nh2, hb2), step2, hs2, 0u);
+        sm100::tmem_st8(s_addr + (c0 >> 1), pk);
+        sm100::tmem_wait_ld_dep16(v1);
+        if (c0 + 32 < 128) sm100::tmem_ld16(s_addr + c0 + 32, v0);
+        const sm100::f2 cp1 = {(float)(c0 + 16), (float)(c0 + 17)};
+        sigmoid_chunk<false>(v1, pk, sm100::fma2(cp1, nh2, hb2), step2, hs2, 0u);
+        sm100::tmem_st8(s_addr + ((c0 + 16) >> 1), pk);
         if (c0 + 32 < 128) sm100::tmem_wait_ld_dep16(v0);
     }
 }
@@ -849,7 +878,11 @@ swat_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (MODE == SWAT_MODE_SIGMOID_) {
                 const float hs = 0.5f * a.scale, hsl = 0.5f * slope;
                 const int rd_w0 = st.i0 + 32 * (warp % 4) - j0;   // first row of this warp
-                act_sigmoid_tile(s_addr, hs, hsl, rd, rd_w0, j0, a.window, a.n_sink);
+                // every pair of the tile in the window: j0 + 127 <= i0 and i0 + 127 - j0 < w
+                if (j0 + 127 <= st.i0 && st.i0 + 127 - j0 < a.window)
+                    act_sigmoid_tile_full(s_addr, hs, hsl, rd);
+                else
+                    act_sigmoid_tile(s_addr, hs, hsl, rd, rd_w0, j0, a.window, a.n_sink);
             } else {
                 const float sc2 = a.scale * LOG2E, sl2 = slope * LOG2E;
                 const float mx = act_softmax_max(s_addr, sc2, sl2, rd, j0, a.window, a.n_sink);
