@@ -149,3 +149,63 @@ def test_full_size_ring_decode_sampled_sequences(wl):
                      slopes=None if sl is None else sl.numpy())
         assert_bf16_close(o[bsel], r, f"{wl.name} step {t}")
         assert torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_decode_per_sequence_positions_ragged_window(mode, d):
+    """Each sequence decodes at its own position ("Sliding Window Attention"
+    glossary, ring-buffer paragraph: slot = pos mod w per sequence): two still
+    inside their first window (only slots with distance <= pos count), two
+    past it (sinks in play), with a window that is not a multiple of the
+    streaming kernel's rows per iteration. GPU and oracle rings take the same
+    fills and steps, so every step compares the same state."""
+    B, H, Hkv, w, s, n_fill = 4, 8, 2, 300, 2, 120
+    base = 1e4 if mode == 0 else 5e5
+    sl = inputs.balanced_alibi_slopes(H) if mode == 0 else None
+    gpu = binding.RingCache(B, H, Hkv, d, w, s, mode=mode, slopes=sl, rope_base=base, device=DEV)
+    ref = oracle.RingCache(B, Hkv, d, w, s, base)
+    f = lambda t: t.float().numpy()
+    kf = inputs.normal((B, n_fill, Hkv, d), 611).to(torch.bfloat16)
+    vf = inputs.normal((B, n_fill, Hkv, d), 612).to(torch.bfloat16)
+    gpu.fill(kf.to(DEV), vf.to(DEV), 0)
+    ref.fill(f(kf), f(vf), 0)
+    offsets = torch.tensor([0, 50, 181, 400], dtype=torch.int64)
+    for t in range(4):
+        q, kn, vn = inputs.decode_step_inputs(B, H, Hkv, d, t)
+        pos = n_fill + t + offsets
+        o = gpu.step(q.to(DEV), kn.to(DEV), vn.to(DEV), pos.to(DEV))
+        _sync_ok()
+        r = ref.step(f(q), f(kn), f(vn), pos.numpy(), mode=mode, slopes=None if sl is None else sl.numpy())
+        assert_bf16_close(o, r, f"step {t} pos {pos.tolist()}")
+
+
+def test_bf16_softmax_decode_steep_scores_rescale():
+    """Softmax decode whose scores climb by ~0.35 per position (RoPE off, keys
+    along q): the running maximum is raised many times inside a split, also
+    by groups whose largest score sits next to masked (not yet written)
+    slots. The "Sliding-window beats linear attention" page's SWA(w, s)
+    softmax over window + sinks is the definition compared against."""
+    B, H, Hkv, d, w, s, n_fill = 2, 8, 2, 128, 300, 2, 200
+    gpu = binding.RingCache(B, H, Hkv, d, w, s, mode=1, slopes=None, rope_base=0.0, device=DEV)
+    ref = oracle.RingCache(B, Hkv, d, w, s, 0.0)
+    f = lambda t: t.float().numpy()
+    kf = torch.zeros(B, n_fill, Hkv, d)
+    kf[..., 0] = 0.1 * torch.arange(n_fill, dtype=torch.float32)[None, :, None]
+    kf = kf.to(torch.bfloat16)
+    vf = inputs.normal((B, n_fill, Hkv, d), 613)
+    gpu.fill(kf.to(DEV), vf.to(DEV), 0)
+    ref.fill(f(kf), f(vf), 0)
+    for t, off in enumerate([0, 150]):
+        pos = torch.full((B,), n_fill + off, dtype=torch.int64)
+        q = torch.zeros(B, H, d)
+        q[..., 0] = 40.0
+        q = q.to(torch.bfloat16)
+        kn = torch.zeros(B, Hkv, d)
+        kn[..., 0] = 0.1 * float(pos[0])
+        kn = kn.to(torch.bfloat16)
+        vn = inputs.normal((B, Hkv, d), 614 + t)
+        o = gpu.step(q.to(DEV), kn.to(DEV), vn.to(DEV), pos.to(DEV))
+        _sync_ok()
+        r = ref.step(f(q), f(kn), f(vn), pos.numpy(), mode=1)
+        assert_bf16_close(o, r, f"pos {int(pos[0])}")

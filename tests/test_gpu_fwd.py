@@ -84,7 +84,11 @@ def test_index_probe_16_tokens_window_4_fp32():
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("N,w,s", [(300, 64, 0), (300, 100, 5), (257, 256, 0), (130, 1, 3), (200, 500, 0)])
+# (257, 256): a 128 x 128 tile whose farthest pair sits at distance 255 is
+# entirely in the window (unmasked pass); (400, 255): at distance 255 it is
+# not, so the same tiles take the masked pass.
+@pytest.mark.parametrize("N,w,s", [(300, 64, 0), (300, 100, 5), (257, 256, 0), (400, 255, 0), (400, 129, 2),
+                                   (130, 1, 3), (200, 500, 0)])
 def test_index_probe_bit_exact(dtype, N, w, s):
     _index_probe(N, w, s, dtype)
 
