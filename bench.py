@@ -42,6 +42,35 @@ def fwd_flops(B, H, d, N, window):
     return 4.0 * B * H * d * band_pairs(N, window)
 
 
+def bwd_traffic_per_call(B):
+    """DRAM bytes (read + write) of one backward call (its dq and dk/dv
+    kernels) at batch B, from the ncu captures summarised in profiles/ (batch
+    4), scaled by B / 4: every unit of work (a 128-row tile of one head) moves
+    the same bytes. None when the kernel source differs from the one captured
+    (its sha256 is recorded in each summary) or a summary is missing."""
+    import hashlib
+    import re
+    src = os.path.join(ROOT, "sliding_window_sigmoid_b200", "csrc", "bwd_tc.cuh")
+    try:
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        total = 0.0
+        for role in ("dq", "dkdv"):
+            with open(os.path.join(ROOT, "profiles", f"swat_bwd_tc_{role}_d64_sigmoid_B4.md")) as f:
+                text = f.read()
+            m = re.search(r"sha256 ([0-9a-f]{64})", text)
+            if not m or m.group(1) != digest:
+                return None
+            for kind in ("read", "write"):
+                b = re.search(r"\| dram__bytes_%s\.sum \| ([0-9.]+) Mbyte \|" % kind, text)
+                if not b:
+                    return None
+                total += float(b.group(1)) * 1e6
+        return total * B / 4.0
+    except OSError:
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -304,7 +333,9 @@ def run_swat(args):
     dom = ("swat_attn_bwd", bwd_ms, bf) if bwd_ms >= fwd_ms else ("swat_attn_fwd", fwd_ms, ff)
     achieved = dom[2] / (dom[1] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": dom[0], "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": bwd_traffic_per_call(B) if dom[0] == "swat_attn_bwd" and d == 64 else None,
+                "traffic_unit": "bytes per call (ncu DRAM read + write, batch-4 captures scaled to the batch)",
                 "peak_source": f"{peak_src} bf16 burst",
                 "fwd": {"tflops": fwd_tf, "frac": fwd_tf / peak, "ms": fwd_ms},
                 "bwd": {"tflops": bwd_tf, "frac": bwd_tf / peak, "ms": bwd_ms}}

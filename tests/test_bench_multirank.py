@@ -72,3 +72,36 @@ def test_two_gloo_ranks_max_seeds_value_and_reference_arm(tmp_path):
     assert line["impl"] == "reference" and line["n_gpus"] == world and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert res[1]["ref_out"] == ""
+
+
+def test_bwd_traffic_from_captures_and_source_hash(tmp_path, monkeypatch):
+    """`traffic` of the backward call: the DRAM bytes of the committed batch-4
+    captures (both kernels) scaled to the batch, and None once the kernel
+    source differs from the captured one."""
+    import re
+    import shutil
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    want = 0.0
+    for role in ("dq", "dkdv"):
+        with open(os.path.join(ROOT, "profiles", f"swat_bwd_tc_{role}_d64_sigmoid_B4.md")) as f:
+            text = f.read()
+        for kind in ("read", "write"):
+            want += float(re.search(r"dram__bytes_%s\.sum \| ([0-9.]+) Mbyte" % kind, text).group(1)) * 1e6
+    assert bench.bwd_traffic_per_call(4) == pytest.approx(want)
+    assert bench.bwd_traffic_per_call(8) == pytest.approx(2 * want)
+    # a copy of the tree whose kernel source changed: no traffic figure
+    (tmp_path / "profiles").mkdir()
+    for role in ("dq", "dkdv"):
+        name = f"swat_bwd_tc_{role}_d64_sigmoid_B4.md"
+        shutil.copy(os.path.join(ROOT, "profiles", name), tmp_path / "profiles" / name)
+    csrc = tmp_path / "sliding_window_sigmoid_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    src = os.path.join(ROOT, "sliding_window_sigmoid_b200", "csrc", "bwd_tc.cuh")
+    shutil.copy(src, csrc / "bwd_tc.cuh")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.bwd_traffic_per_call(8) == pytest.approx(2 * want)
+    with open(csrc / "bwd_tc.cuh", "a") as f:
+        f.write("\n// changed\n")
+    assert bench.bwd_traffic_per_call(8) is None
