@@ -143,15 +143,6 @@ __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap *map, int c0, 
                  : "memory");
 }
 
-// 1-D bulk copy global -> shared (no multicast); 16-byte aligned, size % 16 == 0.
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -320,8 +311,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
 // Wait for outstanding tcgen05.ld and tie the loaded registers to the wait, so
 // the compiler cannot move any use of them above it.
 __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32])
@@ -387,19 +376,6 @@ __device__ __forceinline__ f2 mul2(f2 a, f2 b)
         "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(r.x), "=f"(r.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return r;
-}
-
-// tanh of two values in one MUFU operation (fp16 in and out, ~2^-11 relative):
-// the pair is rounded to f16x2, and the results are returned as fp32.
-__device__ __forceinline__ f2 tanh2_approx_f16(f2 x)
-{
-    uint32_t h, t;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
-    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
-    f2 r;
-    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-        : "=f"(r.x), "=f"(r.y) : "r"(t));
     return r;
 }
 
