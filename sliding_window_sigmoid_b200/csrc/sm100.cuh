@@ -114,7 +114,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
-// TMA (no multicast): 4-D tiled load into shared memory, completing on an mbarrier.
+// TMA: 4-D tiled load into this CTA's shared memory, completing on an mbarrier.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar,
                                             int c0, int c1, int c2, int c3)
