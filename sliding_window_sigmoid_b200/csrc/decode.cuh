@@ -65,11 +65,13 @@ struct FillArgs {
 };
 
 // Writes one raw token (k rotated at position p) into ring slot p mod w and,
-// if p < n_sink, into sink slot p. Threads stride over (kv head, pair).
+// if p < n_sink, into sink slot p. Threads stride over (kv head, pair). The
+// rotation's (cos, sin) of pair t come from cs[t] when given (one table per
+// token, shared by its kv heads), else are computed here.
 template <typename T>
 __device__ void ring_store_token(const T *k_tok, const T *v_tok, T *kc, T *vc, T *ks, T *vs,
                                  int b, int Hkv, int d, int window, int n_sink, long long p,
-                                 bool write_ring, int use_rope, double log2_base)
+                                 bool write_ring, int use_rope, double log2_base, const float2 *cs = nullptr)
 {
     const int half = d / 2;
     const long long slot = p % window;
@@ -79,7 +81,12 @@ __device__ void ring_store_token(const T *k_tok, const T *v_tok, T *kc, T *vc, T
         float y0 = x0, y1 = x1;
         if (use_rope) {
             float c, s;
-            rope_cos_sin(p, rope_theta(t, d, log2_base), c, s);
+            if (cs) {
+                c = cs[t].x;
+                s = cs[t].y;
+            } else {
+                rope_cos_sin(p, rope_theta(t, d, log2_base), c, s);
+            }
             rope_pair(x0, x1, c, s, y0, y1);
         }
         T v0 = v_tok[(size_t)kvh * d + 2 * t], v1 = v_tok[(size_t)kvh * d + 2 * t + 1];
@@ -102,14 +109,24 @@ __device__ void ring_store_token(const T *k_tok, const T *v_tok, T *kc, T *vc, T
 template <typename T>
 __global__ void swa_cache_fill_kernel(FillArgs a)
 {
+    __shared__ float2 cs[64];          // (cos, sin) of p theta_t, d <= 128
     const int t = blockIdx.x, b = blockIdx.y;
     const long long p = a.p0 + t;
     const long long p_end = a.p0 + a.n_tok;
     const bool latest = p + a.window >= p_end;
+    if (!latest && p >= a.n_sink) return;   // overwritten later in the ring, not a sink
+    if (a.use_rope) {
+        for (int i = threadIdx.x; i < a.d / 2; i += blockDim.x) {
+            float c, s;
+            rope_cos_sin(p, rope_theta(i, a.d, a.log2_base), c, s);
+            cs[i] = make_float2(c, s);
+        }
+        __syncthreads();
+    }
     const T *kt = (const T *)a.k + ((size_t)b * a.n_tok + t) * a.Hkv * a.d;
     const T *vt = (const T *)a.v + ((size_t)b * a.n_tok + t) * a.Hkv * a.d;
     ring_store_token<T>(kt, vt, (T *)a.k_cache, (T *)a.v_cache, (T *)a.k_sink, (T *)a.v_sink, b,
-                        a.Hkv, a.d, a.window, a.n_sink, p, latest, a.use_rope, a.log2_base);
+                        a.Hkv, a.d, a.window, a.n_sink, p, latest, a.use_rope, a.log2_base, cs);
 }
 
 // grid (B): the new token of sequence b.
