@@ -5,11 +5,14 @@
 // ring-buffer paragraph: the cache holds the last w keys and values). Each
 // CTA streams DEC_SLOTS_PER_SPLIT consecutive slots of one (b, kv head) for
 // the G query heads that share it, with 16-byte loads: a group of d/8 lanes
-// covers one cache row (each lane owns 8 dimensions), and the loads of
-// several rows are issued before their arithmetic so enough bytes are in
-// flight to cover HBM latency. Split 0 also takes the sink rows. Partial sums
-// (and, in softmax mode, the running maximum and denominator per head) go to
-// the workspace; decode_combine merges them.
+// covers one cache row (each lane owns 8 dimensions), and the loads of four
+// rows per row group are issued before their arithmetic. One thread of the
+// CTA keeps the next DEC_PREFETCH_ITERS iterations of K and V rows (two
+// contiguous ranges) on their way into L2 with bulk prefetches, so those
+// loads mostly hit L2 and the warps need fewer bytes in flight to cover HBM
+// latency. Split 0 also takes the sink rows. Partial sums (and, in softmax
+// mode, the running maximum and denominator per head) go to the workspace;
+// decode_combine merges them.
 #pragma once
 #include "common.cuh"
 #include "decode.cuh"
