@@ -16,14 +16,18 @@
 //   warp 1     TMA producer (one thread): Q tiles, K/V tiles into a ring.
 //   warp 2     schedule (one thread): publishes each step ahead of time in a
 //              shared-memory ring read by the MMA and TMA threads.
-//   warps 4..  activation warpgroup(s) (two in sigmoid mode, taking the steps
-//              in turn): tcgen05.ld S (one query row per thread, TMEM lane =
-//              row), ALiBi term, edge-tile mask, activation, P packed to bf16
-//              and tcgen05.st over the first 64 columns of its S buffer; the
-//              epilogue of each item (O: TMEM -> bf16 global rows).
-//   last 4     RoPE prep: rotate the TMA-staged Q tile and each new K tile in
-//              place in shared memory (SWIZZLE_128B layout), then
-//              fence.proxy.async so the tensor core reads the rotated values.
+//   warps 4..  activation warpgroup(s) (sigmoid mode: two, or three when Q
+//              and K arrive rotated and there are three S buffers, taking the
+//              steps in turn; softmax mode: one): tcgen05.ld S (one query row
+//              per thread, TMEM lane = row), ALiBi term, edge-tile mask (none
+//              for interior tiles, whose pairs are all in the window),
+//              activation, P packed to bf16 and tcgen05.st over the first 64
+//              columns of its S buffer; the epilogue of each item (O: TMEM ->
+//              bf16 global rows).
+//   last 4     RoPE prep (when Q and K are not pre-rotated): rotate the
+//              TMA-staged Q tile and each new K tile in place in shared memory
+//              (SWIZZLE_128B layout), then fence.proxy.async so the tensor
+//              core reads the rotated values.
 // TMEM columns: S buffers [0, 128 NSB), O0 / O1 (double-buffered per item) after them.
 #pragma once
 #include <algorithm>
