@@ -64,9 +64,9 @@ struct FwdTcCfg {
     static constexpr uint32_t COL_O = NSB * 128;              // O0 at COL_O, O1 at COL_O + D
 };
 
-// Warp roles. Sigmoid mode runs two activation warpgroups that take the S
-// tiles in turn (even steps / odd steps), so one computes while the other
-// waits for its next tile; softmax mode keeps one, because a row's running
+// Warp roles. Sigmoid mode runs two or three activation warpgroups that take
+// the S tiles in turn (step % warpgroups), so one computes while the others
+// wait for their next tiles; softmax mode keeps one, because a row's running
 // maximum and sum must live in one thread.
 // Warps 0 and 1 issue MMAs and TMA copies: the scheduler favours older
 // (lower-numbered) warps, and these threads pace everything else. Warp 2
