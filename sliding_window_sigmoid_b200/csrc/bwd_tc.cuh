@@ -17,17 +17,21 @@
 //   DSUM  (softmax) the DQ products without dQ': D_i = sum_j p_ij dP_ij.
 // Each streamed tile is processed as two 64-column half-steps; half-step
 // hs goes to TMEM buffer hs % NBUF and activation warpgroup hs % NWG
-// (NWG = NBUF: 3 for dq at d 64, else 2), so the element-wise pass of one
+// (NWG = NBUF: 3 where three 128-column buffers fit beside the accumulators
+// -- dq, and dk/dv at d 64 -- else 2), so the element-wise pass of one
 // half-step overlaps the MMAs of the next ones.
 // Warp roles (512 threads, one CTA per SM):
 //   warp 0     issues S / dP of each half-step (X MMAs) into its TMEM buffer.
 //   warp 1     TMA: stationary tile pair per item, streamed pairs into a ring.
 //   warp 3     issues the gradient MMAs (dV, dK', dQ') of each half-step.
 //   warps 4..  NWG activation warpgroups (one TMEM lane = one row per
-//              thread); the epilogue of an item runs in one of them,
-//              deferred until after its next half-step.
+//              thread); the epilogue of an item runs in one of them:
+//              deferred until after its next half-step where two
+//              accumulator sets fit, else right after the item's last
+//              half-step, releasing the accumulators after its last TMEM load.
 //   others     set-up only. Q and K arrive RoPE-rotated: a small kernel
-//              writes rotated copies into the workspace first.
+//              writes rotated copies into the workspace first, or the
+//              forward's copies are reused (swat_attn_bwd_rotated).
 // TMEM columns: buffer b = [128 b, 128 b + 128): S half, then dP half (bf16
 // P and dS over their first 32 columns, or in columns of their own);
 // accumulators after the buffers.
