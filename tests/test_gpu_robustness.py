@@ -50,9 +50,13 @@ def _sync_ok():
     assert binding.device_status() == 0
 
 
-@pytest.mark.parametrize("mode,N,d,w,s", [(0, 300, 64, 64, 0), (0, 333, 128, 200, 0), (1, 300, 64, 100, 3)])
-def test_forward_backward_write_only_their_tensors(mode, N, d, w, s):
-    B, H, Hkv = 2, 4, 2
+@pytest.mark.parametrize("mode,H,Hkv,N,d,w,s", [
+    (0, 4, 2, 300, 64, 64, 0),       # sigmoid, GQA, d 64
+    (0, 4, 2, 333, 128, 200, 0),     # sigmoid, GQA, d 128
+    (1, 8, 2, 300, 128, 64, 4),      # SWA(64, 4) shape: softmax with sinks, GQA
+])
+def test_forward_backward_write_only_their_tensors(mode, H, Hkv, N, d, w, s):
+    B = 2
     scale = 1.0 / np.sqrt(d) if mode == 0 else 1.0
     q, k, v, do = [t.to(DEV) for t in inputs.qkv(B, N, H, Hkv, d, seed=31, scale=scale, dtype=torch.bfloat16,
                                                   with_dout=True)]
@@ -98,7 +102,7 @@ def test_forward_backward_deterministic(mode):
     B, H, Hkv, N, d, w = 2, 4, 4, 700, 64, 256
     q, k, v, do = [t.to(DEV) for t in inputs.qkv(B, N, H, Hkv, d, seed=32, scale=0.125, dtype=torch.bfloat16,
                                                   with_dout=True)]
-    kw = dict(window=w, n_sink=2 if mode == 1 else 0, mode=mode,
+    kw = dict(window=w, n_sink=0, mode=mode,
               slopes=inputs.balanced_alibi_slopes(H) if mode == 0 else None, rope_base=1e4)
     runs = []
     for _ in range(2):
